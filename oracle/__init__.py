@@ -1,0 +1,182 @@
+"""fp64 CPU oracle for scaled-dot-product attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+leg of ``bench.py`` may import this package.  The product library never does,
+and this package imports nothing from the product.
+
+The arithmetic lives in ``sdpa_oracle.c`` (plain C, fp64, no fast-math); this
+module compiles it with gcc on first use and wraps it with ctypes.  Every
+function takes and returns numpy float64 arrays in the [B, H, S, d] layout.
+
+Sources followed (page title and section):
+  * "PyTorch attention profiling: Flash, cuDNN, Math backends", section 1
+    (naive attention, five steps) and "math backend" (_safe_softmax)
+      -> attn_fwd, attn_rows
+  * "FlashAttention-2" notes, "algorithm overview" (online-softmax loop)
+      -> online_attn  (used only as a pin of the plain definition)
+  * "[onnxruntime] WebGPU FlashAttention: kernel fusion ...", section 1
+    (fused decode partial with (max, sum) metadata, VxReduce rescale)
+      -> split_partials, split_combine
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sdpa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libsdpa_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+CAUSAL_NONE, CAUSAL_TOP_LEFT, CAUSAL_BOTTOM_RIGHT = 0, 1, 2
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I64 = ctypes.POINTER(ctypes.c_int64)
+_I32 = ctypes.POINTER(ctypes.c_int)
+
+
+def build(force: bool = False) -> str:
+    """Compile sdpa_oracle.c into libsdpa_oracle.so (gcc, -O2, no fast-math)."""
+    stale = (not os.path.exists(_LIB_PATH)) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", "-O2", "-std=c11", "-fno-fast-math", "-shared", "-fPIC",
+                        "-pthread", _SRC, "-o", tmp, "-lm"], check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def bind(lib):
+    """Declare the C signatures on a loaded copy of the oracle library."""
+    i, d = ctypes.c_int, ctypes.c_double
+    lib.oracle_attn_fwd.argtypes = [_D, _D, _D, _D, _D, i, i, i, i, i, i, d, i, i]
+    lib.oracle_attn_rows.argtypes = [_D, _D, _D, i, i, i, i, i, i, d, i,
+                                     _I64, ctypes.c_int64, _D, _D, i]
+    lib.oracle_online_attn.argtypes = [_D, _D, _D, _D, _D, i, i, i, i, i, i, d, i, i, i]
+    lib.oracle_split_partials.argtypes = [_D, _D, _D, i, i, i, i, i, i, d, i,
+                                          _I32, i, _D, _D, _D]
+    lib.oracle_split_combine.argtypes = [_D, _D, _D, ctypes.c_int64, i, i, _D, _D]
+    for f in (lib.oracle_attn_fwd, lib.oracle_attn_rows, lib.oracle_online_attn,
+              lib.oracle_split_partials, lib.oracle_split_combine):
+        f.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    return a
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(_D)
+
+
+def _dims(q, k, v):
+    B, Hq, Sq, d = q.shape
+    Bk, Hkv, Sk, dk = k.shape
+    if Bk != B or dk != d:
+        raise ValueError("q and k disagree on batch or head_dim")
+    if v.shape != k.shape:
+        raise ValueError("v must have the shape of k")
+    return B, Hq, Hkv, Sq, Sk, d
+
+
+def _threads(nthreads):
+    return int(nthreads) if nthreads else (os.cpu_count() or 1)
+
+
+def attn_fwd(q, k, v, scale: float, causal: int = CAUSAL_NONE, nthreads: int | None = None):
+    """The five naive steps for every row.  Returns (o[B,Hq,Sq,d], lse[B,Hq,Sq])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Hkv, Sq, Sk, d = _dims(q, k, v)
+    o = np.zeros((B, Hq, Sq, d))
+    lse = np.zeros((B, Hq, Sq))
+    st = _load().oracle_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                 B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal),
+                                 _threads(nthreads))
+    if st != 0:
+        raise ValueError(f"oracle_attn_fwd failed ({st})")
+    return o, lse
+
+
+def attn_rows(q, k, v, scale: float, causal: int, rows, nthreads: int | None = None):
+    """The five naive steps for selected rows.
+
+    ``rows`` are flattened indices (b*Hq + hq)*Sq + i.  Returns (o[n,d], lse[n]).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Hkv, Sq, Sk, d = _dims(q, k, v)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    n = rows.shape[0]
+    o = np.zeros((n, d))
+    lse = np.zeros((n,))
+    st = _load().oracle_attn_rows(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Sq, Sk, d,
+                                  float(scale), int(causal), rows.ctypes.data_as(_I64), n,
+                                  _ptr(o), _ptr(lse), _threads(nthreads))
+    if st != 0:
+        raise ValueError(f"oracle_attn_rows failed ({st})")
+    return o, lse
+
+
+def online_attn(q, k, v, scale: float, causal: int, block_q: int, block_k: int):
+    """The FlashAttention-2 online-softmax recurrence in fp64 (a pin, not a product)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Hkv, Sq, Sk, d = _dims(q, k, v)
+    o = np.zeros((B, Hq, Sq, d))
+    lse = np.zeros((B, Hq, Sq))
+    st = _load().oracle_online_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                    B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal),
+                                    int(block_q), int(block_k))
+    if st != 0:
+        raise ValueError(f"oracle_online_attn failed ({st})")
+    return o, lse
+
+
+def split_partials(q, k, v, scale: float, causal: int, bounds):
+    """Per-split locally normalised partials and (max, sum) metadata.
+
+    ``bounds`` is a list [0, b1, ..., Sk] of split boundaries over the keys.
+    Returns (part_o[B,Hq,Sq,ns,d], part_m[B,Hq,Sq,ns], part_l[B,Hq,Sq,ns]).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Hkv, Sq, Sk, d = _dims(q, k, v)
+    b = np.ascontiguousarray(np.asarray(bounds, dtype=np.int32))
+    ns = b.shape[0] - 1
+    po = np.zeros((B, Hq, Sq, ns, d))
+    pm = np.zeros((B, Hq, Sq, ns))
+    pl = np.zeros((B, Hq, Sq, ns))
+    st = _load().oracle_split_partials(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Sq, Sk, d,
+                                       float(scale), int(causal), b.ctypes.data_as(_I32), ns,
+                                       _ptr(po), _ptr(pm), _ptr(pl))
+    if st != 0:
+        raise ValueError(f"oracle_split_partials failed ({st})")
+    return po, pm, pl
+
+
+def split_combine(part_o, part_m, part_l):
+    """Combine split partials.  part_o is [..., ns, d]; returns (o[..., d], lse[...])."""
+    po, pm, pl = _f64(part_o), _f64(part_m), _f64(part_l)
+    lead = po.shape[:-2]
+    ns, d = po.shape[-2], po.shape[-1]
+    n = int(np.prod(lead)) if lead else 1
+    o = np.zeros(lead + (d,))
+    lse = np.zeros(lead)
+    st = _load().oracle_split_combine(_ptr(po), _ptr(pm), _ptr(pl), n, ns, d,
+                                      _ptr(o), _ptr(lse))
+    if st != 0:
+        raise ValueError(f"oracle_split_combine failed ({st})")
+    return o, lse

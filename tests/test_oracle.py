@@ -1,0 +1,307 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+None of these re-types the oracle's formula: each one checks a closed form,
+an invariant, a hand-derived example or an independent brute force, chosen so
+that a dropped term, a wrong sign or index, a transposed operand, a wrong
+causal alignment or a wrong GQA mapping fails at least one of them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_worked.json")
+NONE, TL, BR = 0, 1, 2
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def _visible(causal, i, j, Sq, Sk):
+    if causal == TL:
+        return j <= i
+    if causal == BR:
+        return j <= i + Sk - Sq
+    return True
+
+
+def brute_force(q, k, v, scale, causal):
+    """Independent scalar attention: nested loops, math.exp, math.fsum, no max
+    subtraction (inputs are tiny, so exp cannot overflow)."""
+    B, Hq, Sq, d = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    o = [[[[0.0] * d for _ in range(Sq)] for _ in range(Hq)] for _ in range(B)]
+    lse = [[[0.0] * Sq for _ in range(Hq)] for _ in range(B)]
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // G
+            for i in range(Sq):
+                w = []
+                for j in range(Sk):
+                    if not _visible(causal, i, j, Sq, Sk):
+                        continue
+                    x = scale * math.fsum(float(q[b, h, i, c]) * float(k[b, hk, j, c])
+                                          for c in range(d))
+                    w.append((j, math.exp(x)))
+                if not w:
+                    lse[b][h][i] = -math.inf
+                    continue
+                z = math.fsum(e for _, e in w)
+                lse[b][h][i] = math.log(z)
+                for c in range(d):
+                    o[b][h][i][c] = math.fsum(e * float(v[b, hk, j, c]) for j, e in w) / z
+    return np.array(o), np.array(lse)
+
+
+# ------------------------------------------------------------ hand-worked
+
+def _ev(x):
+    return float(eval(x, {"__builtins__": {}}, {"log": math.log, "inf": math.inf}))
+
+
+def _arr(nested):
+    if isinstance(nested, list):
+        return [_arr(x) for x in nested]
+    return _ev(nested)
+
+
+@pytest.mark.parametrize("case", json.load(open(GOLDEN))["cases"], ids=lambda c: c["name"])
+def test_hand_worked_examples(oracle_mod, case):
+    q, k, v = (np.array(_arr(case[n])) for n in ("q", "k", "v"))
+    o_exp, lse_exp = np.array(_arr(case["o"])), np.array(_arr(case["lse"]))
+    o, lse = oracle_mod.attn_fwd(q, k, v, _ev(case["scale"]), case["causal"])
+    np.testing.assert_allclose(o, o_exp, rtol=0, atol=1e-12)
+    assert np.array_equal(np.isneginf(lse), np.isneginf(lse_exp))
+    fin = np.isfinite(lse_exp)
+    np.testing.assert_allclose(lse[fin], lse_exp[fin], rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------ brute force
+
+TINY_SHAPES = list(itertools.product((1, 2, 3, 4), (1, 2, 3, 4), (1, 2, 3, 4), (1, 2),
+                                     (NONE, TL, BR)))
+
+
+def test_brute_force_every_tiny_shape(oracle_mod):
+    """Every Sq, Sk in 1..4, d in 1..4, group size 1 or 2, each causal mode."""
+    for n, (Sq, Sk, d, G, causal) in enumerate(TINY_SHAPES):
+        Hkv = 2
+        Hq = Hkv * G
+        q = _rand((2, Hq, Sq, d), 10 * n)
+        k = _rand((2, Hkv, Sk, d), 10 * n + 1)
+        v = _rand((2, Hkv, Sk, d), 10 * n + 2)
+        scale = 1.0 / math.sqrt(d)
+        o, lse = oracle_mod.attn_fwd(q, k, v, scale, causal)
+        ob, lseb = brute_force(q, k, v, scale, causal)
+        assert not np.isnan(o).any()
+        np.testing.assert_allclose(o, ob, rtol=0, atol=1e-12,
+                                   err_msg=f"Sq={Sq} Sk={Sk} d={d} G={G} causal={causal}")
+        assert np.array_equal(np.isneginf(lse), np.isneginf(lseb))
+        fin = np.isfinite(lseb)
+        np.testing.assert_allclose(lse[fin], lseb[fin], rtol=0, atol=1e-12)
+
+
+def test_probabilities_sum_to_one_and_match_exp(oracle_mod):
+    """With v = identity (d = Sk) the output row IS the softmax row: it must sum
+    to 1, vanish on masked keys and be proportional to exp(scale * q.k)."""
+    Sk = 24
+    Sq = 20
+    for causal in (NONE, TL, BR):
+        q = _rand((1, 1, Sq, Sk), 3)
+        k = _rand((1, 1, Sk, Sk), 4)
+        v = np.eye(Sk)[None, None]
+        scale = 0.3
+        p, lse = oracle_mod.attn_fwd(q, k, v, scale, causal)
+        p = p[0, 0]
+        np.testing.assert_allclose(p.sum(-1), 1.0, rtol=0, atol=1e-12)
+        x = scale * (q[0, 0] @ k[0, 0].T)
+        for i in range(Sq):
+            vis = np.array([_visible(causal, i, j, Sq, Sk) for j in range(Sk)])
+            assert np.all(p[i, ~vis] == 0.0)
+            np.testing.assert_allclose(p[i, vis], np.exp(x[i, vis] - lse[0, 0, i]),
+                                       rtol=1e-12, atol=0)
+
+
+# ----------------------------------------------------- closed forms / invariants
+
+def test_causal_row0_is_v0(oracle_mod):
+    q = _rand((2, 3, 50, 16), 5)
+    k = _rand((2, 3, 50, 16), 6)
+    v = _rand((2, 3, 50, 16), 7)
+    o, lse = oracle_mod.attn_fwd(q, k, v, 0.25, TL)
+    assert np.array_equal(o[:, :, 0, :], v[:, :, 0, :])
+    np.testing.assert_allclose(lse[:, :, 0], 0.25 * np.einsum("bhd,bhd->bh", q[:, :, 0], k[:, :, 0]),
+                               rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [NONE, TL, BR])
+def test_zero_query_gives_prefix_mean(oracle_mod, causal):
+    """q = 0 makes every score 0: each row averages the V rows it may see and
+    lse = log(count)."""
+    Sq, Sk, d = 37, 53, 8
+    if causal == TL:
+        Sq = Sk  # keep every row non-empty
+    q = np.zeros((1, 2, Sq, d))
+    k = _rand((1, 2, Sk, d), 8)
+    v = _rand((1, 2, Sk, d), 9)
+    o, lse = oracle_mod.attn_fwd(q, k, v, 0.7, causal)
+    for i in range(Sq):
+        cnt = sum(_visible(causal, i, j, Sq, Sk) for j in range(Sk))
+        np.testing.assert_allclose(o[:, :, i], v[:, :, :cnt].mean(axis=2), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[:, :, i], math.log(cnt), rtol=0, atol=1e-12)
+
+
+def test_single_key_returns_v0(oracle_mod):
+    q = _rand((2, 2, 9, 32), 10)
+    k = _rand((2, 2, 1, 32), 11)
+    v = _rand((2, 2, 1, 32), 12)
+    o, _ = oracle_mod.attn_fwd(q, k, v, 0.1, NONE)
+    np.testing.assert_allclose(o, np.broadcast_to(v, o.shape), rtol=0, atol=1e-15)
+
+
+def test_identical_keys_give_mean_of_visible_v(oracle_mod):
+    Sq = Sk = 31
+    q = _rand((1, 1, Sq, 8), 13) * 5.0
+    k = np.broadcast_to(_rand((1, 1, 1, 8), 14), (1, 1, Sk, 8)).copy()
+    v = _rand((1, 1, Sk, 8), 15)
+    o, _ = oracle_mod.attn_fwd(q, k, v, 1.0, TL)
+    for i in range(Sq):
+        np.testing.assert_allclose(o[0, 0, i], v[0, 0, :i + 1].mean(axis=0), rtol=0, atol=1e-12)
+
+
+def test_noncausal_permutation_invariance(oracle_mod):
+    q = _rand((1, 2, 17, 16), 16)
+    k = _rand((1, 2, 40, 16), 17)
+    v = _rand((1, 2, 40, 16), 18)
+    perm = np.random.default_rng(0).permutation(40)
+    o1, l1 = oracle_mod.attn_fwd(q, k, v, 0.25, NONE)
+    o2, l2 = oracle_mod.attn_fwd(q, k[:, :, perm], v[:, :, perm], 0.25, NONE)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-12)
+
+
+def test_score_shift_invariance(oracle_mod):
+    """Append a dimension with q=1 and k=c: every score moves by scale*c, so O is
+    unchanged and lse moves by scale*c."""
+    q = _rand((1, 1, 12, 8), 19)
+    k = _rand((1, 1, 12, 8), 20)
+    v = _rand((1, 1, 12, 8), 21)
+    c, scale = 3.5, 0.5
+    q2 = np.concatenate([q, np.ones((1, 1, 12, 1))], axis=-1)
+    k2 = np.concatenate([k, np.full((1, 1, 12, 1), c)], axis=-1)
+    v2 = np.concatenate([v, np.zeros((1, 1, 12, 1))], axis=-1)
+    for causal in (NONE, TL):
+        o1, l1 = oracle_mod.attn_fwd(q, k, v, scale, causal)
+        o2, l2 = oracle_mod.attn_fwd(q2, k2, v2, scale, causal)
+        np.testing.assert_allclose(o1, o2[..., :8], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l1 + scale * c, l2, rtol=0, atol=1e-12)
+
+
+def test_scale_multiplies_scores(oracle_mod):
+    q = _rand((1, 2, 10, 8), 22)
+    k = _rand((1, 2, 10, 8), 23)
+    v = _rand((1, 2, 10, 8), 24)
+    o1, l1 = oracle_mod.attn_fwd(q, k, v, 2.0, TL)
+    o2, l2 = oracle_mod.attn_fwd(2.0 * q, k, v, 1.0, TL)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [NONE, TL, BR])
+def test_gqa_equals_explicit_expansion(oracle_mod, causal):
+    Hq, Hkv = 8, 2
+    q = _rand((2, Hq, 11, 8), 25)
+    k = _rand((2, Hkv, 14, 8), 26)
+    v = _rand((2, Hkv, 14, 8), 27)
+    o1, l1 = oracle_mod.attn_fwd(q, k, v, 0.3, causal)
+    G = Hq // Hkv
+    o2, l2 = oracle_mod.attn_fwd(q, np.repeat(k, G, axis=1), np.repeat(v, G, axis=1), 0.3, causal)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+    # and a wrong mapping (hq % Hkv) would differ
+    o3, _ = oracle_mod.attn_fwd(q, np.tile(k, (1, G, 1, 1)), np.tile(v, (1, G, 1, 1)), 0.3, causal)
+    assert np.abs(o1 - o3).max() > 1e-3
+
+
+def test_rows_api_matches_full(oracle_mod):
+    q = _rand((2, 4, 19, 16), 28)
+    k = _rand((2, 2, 23, 16), 29)
+    v = _rand((2, 2, 23, 16), 30)
+    o, lse = oracle_mod.attn_fwd(q, k, v, 0.25, BR)
+    rows = np.array([0, 5, 18, 19, 75, 2 * 4 * 19 - 1])
+    orow, lrow = oracle_mod.attn_rows(q, k, v, 0.25, BR, rows)
+    np.testing.assert_array_equal(orow, o.reshape(-1, 16)[rows])
+    np.testing.assert_array_equal(lrow, lse.reshape(-1)[rows])
+
+
+# ------------------------------------------------------- FA2 recurrence pin
+
+@pytest.mark.parametrize("bk", [1, 3, 128])
+@pytest.mark.parametrize("causal", [NONE, TL, BR])
+def test_online_recurrence_equals_definition(oracle_mod, causal, bk):
+    """The FlashAttention-2 loop (running max/sum, one final division) reaches
+    the plain five-step result for any key-block size."""
+    q = _rand((1, 2, 45, 16), 31) * 2.0
+    k = _rand((1, 2, 70, 16), 32) * 2.0
+    v = _rand((1, 2, 70, 16), 33)
+    o1, l1 = oracle_mod.attn_fwd(q, k, v, 0.4, causal)
+    o2, l2 = oracle_mod.online_attn(q, k, v, 0.4, causal, block_q=7, block_k=bk)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------- split-KV combine pin
+
+def _bounds(Sk, ns):
+    return [round(s * Sk / ns) for s in range(ns + 1)]
+
+
+@pytest.mark.parametrize("ns", [1, 2, 3, 7, 61])
+@pytest.mark.parametrize("causal", [NONE, BR])
+def test_split_combine_equals_unsplit(oracle_mod, ns, causal):
+    """Locally normalised partials rescaled by their (max, sum) metadata give
+    exactly full softmax.V (the decode reduce step)."""
+    Sq, Sk = 4, 61
+    q = _rand((2, 8, Sq, 16), 34) * 2.0
+    k = _rand((2, 2, Sk, 16), 35) * 2.0
+    v = _rand((2, 2, Sk, 16), 36)
+    o1, l1 = oracle_mod.attn_fwd(q, k, v, 0.35, causal)
+    po, pm, pl = oracle_mod.split_partials(q, k, v, 0.35, causal, _bounds(Sk, ns))
+    o2, l2 = oracle_mod.split_combine(po, pm, pl)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-12)
+
+
+def test_split_with_masked_and_empty_splits(oracle_mod):
+    """Bottom-right mask with Sq > Sk: some splits see nothing (weight 0) and
+    some rows see nothing at all (o = 0, lse = -inf)."""
+    Sq, Sk = 9, 6
+    q = _rand((1, 2, Sq, 8), 37)
+    k = _rand((1, 1, Sk, 8), 38)
+    v = _rand((1, 1, Sk, 8), 39)
+    o1, l1 = oracle_mod.attn_fwd(q, k, v, 0.5, BR)
+    po, pm, pl = oracle_mod.split_partials(q, k, v, 0.5, BR, [0, 2, 2, 5, 6])
+    assert (pl == 0).any()
+    o2, l2 = oracle_mod.split_combine(po, pm, pl)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-12)
+    assert np.array_equal(np.isneginf(l1), np.isneginf(l2))
+    assert np.isneginf(l1).any() and not np.isnan(o1).any()
+    fin = np.isfinite(l1)
+    np.testing.assert_allclose(l1[fin], l2[fin], rtol=0, atol=1e-12)
+
+
+def test_partials_are_locally_normalised(oracle_mod):
+    """Each split's partial is softmax over that split's keys alone (the fused
+    decode kernel's local normalisation)."""
+    q = _rand((1, 1, 1, 8), 40)
+    k = _rand((1, 1, 10, 8), 41)
+    v = _rand((1, 1, 10, 8), 42)
+    po, pm, pl = oracle_mod.split_partials(q, k, v, 0.5, NONE, [0, 4, 10])
+    o_a, l_a = oracle_mod.attn_fwd(q, k[:, :, :4], v[:, :, :4], 0.5, NONE)
+    np.testing.assert_allclose(po[0, 0, 0, 0], o_a[0, 0, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(pm[0, 0, 0, 0] + math.log(pl[0, 0, 0, 0]), l_a[0, 0, 0], atol=1e-12)

@@ -1,0 +1,67 @@
+"""The pins must catch plausible mistakes in the oracle.
+
+Each case plants one mistake in a private copy of the oracle's C source (a
+dropped term, a wrong sign or index, a wrong mask alignment, a wrong GQA map),
+compiles it on the CPU, swaps it in, and checks that the pin suite fails.
+The real oracle is restored afterwards.
+"""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "sdpa_oracle.c")
+
+MUTATIONS = {
+    "drop_scale": ("for (int j = 0; j < Sk; ++j) scores[j] *= a->scale;", ""),
+    "strict_top_left": ("if (causal == 1) return j <= i;", "if (causal == 1) return j < i;"),
+    "bottom_right_offset_sign": ("return j <= i + (Sk - Sq);", "return j <= i + (Sq - Sk);"),
+    "gqa_modulo_map": ("const int hk = hq / group;\n    const double *qrow",
+                       "const int hk = hq % a->Hkv;\n    const double *qrow"),
+    "no_normalisation": ("for (int j = 0; j < Sk; ++j) scores[j] /= sum;", ""),
+    "lse_without_max": ("*lse_out = mx + log(sum);", "*lse_out = log(sum);"),
+    "reversed_v_rows": ("const double *vrow = vbase + (size_t)j * d;",
+                        "const double *vrow = vbase + (size_t)(Sk - 1 - j) * d;"),
+    "combine_drops_local_sum": ("const double w = ls * exp(part_m[r * ns + s] - M);",
+                                "const double w = exp(part_m[r * ns + s] - M);"),
+    "partials_not_local_max": ("const double p = exp(x[j] - mx);", "const double p = exp(x[j]);"),
+}
+
+
+def _pin_suite(mod):
+    """Run the pins that need no pytest parametrisation machinery."""
+    import json
+    for case in json.load(open(pins.GOLDEN))["cases"]:
+        pins.test_hand_worked_examples(mod, case)
+    pins.test_brute_force_every_tiny_shape(mod)
+    for causal in (0, 1, 2):
+        pins.test_gqa_equals_explicit_expansion(mod, causal)
+    for ns in (2, 3):
+        for causal in (0, 2):
+            pins.test_split_combine_equals_unsplit(mod, ns, causal)
+    pins.test_split_with_masked_and_empty_splits(mod)
+    pins.test_partials_are_locally_normalised(mod)
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(tmp_path, monkeypatch, name):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not unique"
+    mutated = tmp_path / "mutant.c"
+    mutated.write_text(src.replace(old, new))
+    so = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-shared", "-fPIC", "-pthread", str(mutated),
+                    "-o", str(so), "-lm"], check=True)
+    monkeypatch.setattr(oracle, "_lib", oracle.bind(ctypes.CDLL(str(so))))
+    with pytest.raises(AssertionError):
+        _pin_suite(oracle)
+
+
+def test_unmutated_oracle_passes_suite():
+    oracle._lib = None
+    _pin_suite(oracle)
