@@ -1,0 +1,473 @@
+"""Benchmark of the fused attention forward on B200 (one JSON line on rank 0).
+
+Step = one pass of the non-causal d=128 prefill sweep over a 16k-token batch
+(H=16; seq 512, 1024, 2048, 4096 with B = 16384/seq), each shape one
+``attn_fwd`` call through the C ABI, inputs resident in HBM, L2 flushed (a
+256 MiB write) before every call.  ``value`` is TFLOP/s = algorithmic FLOPs
+(4*B*H*S*S*d per shape) / summed CUDA-event time of the calls, max over ranks.
+The other workloads (causal sweep, GQA long sequence, split-KV decode) are
+measured in the same run and reported under ``breakdown``.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch under torchrun; every rank runs the same per-GPU work
+(weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from scaled_dot_product_fa2_b200 import inputs  # noqa: E402
+
+HEADLINE = inputs.PREFILL_NONCAUSAL
+METRIC = "attn fwd TFLOP/s (bf16, d=128) and decode KV GB/s, as fraction of B200 roofline"
+L2_FLUSH_BYTES = 256 << 20
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "prefill_traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-breakdown", action="store_true", help="time the headline step only")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "scaled_dot_product_fa2_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload_name: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        t = json.load(f)
+    if t.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return t.get("per_launch_bytes", {}).get(workload_name)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def setup_dist(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device(f"cuda:{local}"))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, x: float) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+class CpuOracleSample:
+    """Times the oracle (as it stands) on bounded random row samples of a
+    workload, on all host cores."""
+
+    def __init__(self, w):
+        import numpy as np
+        self.np = np
+        self.w = w
+        q, k, v = inputs.workload_inputs(w)
+        self.qd, self.kd, self.vd = q.double().numpy(), k.double().numpy(), v.double().numpy()
+        self.threads = os.cpu_count() or 1
+        self.rng = np.random.default_rng(0)
+        self.total_rows = w.B * w.Hq * w.Sq
+        self.per_row = None
+
+    def _flops(self, rows):
+        w, np = self.w, self.np
+        i = rows % w.Sq
+        if w.causal == inputs.CAUSAL_TOP_LEFT:
+            keys = np.minimum(i + 1, w.Sk)
+        elif w.causal == inputs.CAUSAL_BOTTOM_RIGHT:
+            keys = np.clip(i + w.Sk - w.Sq + 1, 0, w.Sk)
+        else:
+            keys = np.full_like(i, w.Sk)
+        return float(4.0 * w.d * keys.sum())
+
+    def _run(self, n):
+        import oracle
+        rows = self.np.sort(self.rng.choice(self.total_rows, size=n, replace=False))
+        t0 = time.perf_counter()
+        oracle.attn_rows(self.qd, self.kd, self.vd, self.w.eff_scale, self.w.causal, rows, nthreads=self.threads)
+        return rows, time.perf_counter() - t0
+
+    def sample(self, target_s: float):
+        """Returns (TFLOP/s, threads, description, seconds) for about target_s of work."""
+        if self.per_row is None:
+            n = min(self.total_rows, 8 * self.threads)
+            _, dt = self._run(n)
+            self.per_row = dt / n
+        n = int(min(self.total_rows, max(self.threads, target_s / max(self.per_row, 1e-9))))
+        rows, dt = self._run(n)
+        tflops = self._flops(rows) / dt / 1e12
+        desc = (f"{n} random query rows of {self.w.name} (of {self.total_rows}), fp64 oracle on "
+                f"{self.threads} threads, {dt:.1f} s")
+        return tflops, self.threads, desc, dt
+
+
+# ------------------------------------------------------------------ GPU timing
+
+class GpuPrefill:
+    def __init__(self, w, rank: int):
+        q, k, v = inputs.make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Sk, w.d, w.seed + 7919 * rank)
+        self.w = w
+        self.host = [t.pin_memory() for t in (q, k, v)]
+        self.q, self.k, self.v = (t.cuda() for t in (q, k, v))
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device="cuda")
+        self.o_host = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.lse_host = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
+
+    def run(self):
+        import scaled_dot_product_fa2_b200 as sdpa
+        sdpa.attn_fwd(self.q, self.k, self.v, causal=self.w.causal, scale=self.w.scale, out=self.o, lse=self.lse)
+
+    def run_e2e(self):
+        import scaled_dot_product_fa2_b200 as sdpa
+        self.q.copy_(self.host[0], non_blocking=True)
+        self.k.copy_(self.host[1], non_blocking=True)
+        self.v.copy_(self.host[2], non_blocking=True)
+        sdpa.attn_fwd(self.q, self.k, self.v, causal=self.w.causal, scale=self.w.scale, out=self.o, lse=self.lse)
+        self.o_host.copy_(self.o, non_blocking=True)
+        self.lse_host.copy_(self.lse, non_blocking=True)
+
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in self.host)
+
+    def d2h_bytes(self):
+        return self.o.numel() * 2 + self.lse.numel() * 4
+
+
+class GpuDecode:
+    def __init__(self, w, rank: int, copies: int = 3):
+        import scaled_dot_product_fa2_b200 as sdpa
+        self.w = w
+        q, k, v = inputs.make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Sk, w.d, w.seed + 7919 * rank)
+        self.q = q.cuda()
+        # several cache copies (3 x 256 MiB > L2) so each call streams from HBM
+        self.kv = []
+        for c in range(copies):
+            kk, vv = k.cuda(), v.cuda()
+            if c:
+                kk = kk.clone()
+                vv = vv.clone()
+            self.kv.append((kk, vv))
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device="cuda")
+        self.ws = sdpa.decode_workspace(self.q, self.kv[0][0])
+        self.i = 0
+
+    def run(self):
+        import scaled_dot_product_fa2_b200 as sdpa
+        k, v = self.kv[self.i % len(self.kv)]
+        self.i += 1
+        sdpa.attn_decode_splitkv(self.q, k, v, causal=self.w.causal, scale=self.w.scale, workspace=self.ws,
+                                 out=self.o, lse=self.lse)
+
+
+def timed_calls(fns, flush, reps: int, warmup: int):
+    """Per-call CUDA-event times (ms) on the current stream, L2 flushed before each call."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        for fn in fns:
+            flush()
+            fn()
+    torch.cuda.synchronize()
+    times = [[] for _ in fns]
+    for _ in range(reps):
+        for i, fn in enumerate(fns):
+            flush()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            times[i].append((a, b))
+    torch.cuda.synchronize()
+    return [[a.elapsed_time(b) for a, b in ts] for ts in times]
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        # the CPU oracle arm needs no process group: rank 0 runs, the others exit
+        return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+    world, rank, local = setup_dist(args)
+    import scaled_dot_product_fa2_b200 as sdpa
+    from scaled_dot_product_fa2_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(world)
+    peaks, peaks_kind = load_peaks()
+
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = lambda: flush_buf.fill_(1)  # noqa: E731
+
+    shapes = [GpuPrefill(w, rank) for w in HEADLINE]
+    flops_step = sum(s.w.flops() for s in shapes)
+
+    # warm-up (untimed)
+    for _ in range(max(args.warmup, 3)):
+        for s in shapes:
+            flush()
+            s.run()
+    sdpa.check_device_error()
+
+    # ---- timed region: exactly K steps, barrier + synchronize on both sides
+    stream = torch.cuda.current_stream()
+    events = []
+    with ClockSampler(local) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        wall0 = time.perf_counter()
+        for _ in range(args.steps):
+            for s in shapes:
+                flush()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                s.run()
+                b.record(stream)
+                events.append((s.w.name, a, b))
+        torch.cuda.synchronize()
+        barrier(world)
+        wall = time.perf_counter() - wall0
+    sdpa.check_device_error()
+    per_shape_ms = {}
+    for name, a, b in events:
+        per_shape_ms.setdefault(name, []).append(a.elapsed_time(b))
+    kernel_ms = sum(sum(v) for v in per_shape_ms.values())
+    kernel_ms = max_over_ranks(world, kernel_ms)
+    wall = max_over_ranks(world, wall)
+    ms_per_step = kernel_ms / args.steps
+    value = world * flops_step * args.steps / (kernel_ms / 1e3) / 1e12
+
+    # ---- end to end through the public API with host buffers (pinned), same metric
+    for _ in range(2):
+        for s in shapes:
+            s.run_e2e()
+    torch.cuda.synchronize()
+    barrier(world)
+    e_a = torch.cuda.Event(enable_timing=True)
+    e_b = torch.cuda.Event(enable_timing=True)
+    e_a.record(stream)
+    for _ in range(args.steps):
+        for s in shapes:
+            s.run_e2e()
+    e_b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(world, e_a.elapsed_time(e_b))
+    e2e_value = world * flops_step * args.steps / (e2e_ms / 1e3) / 1e12
+    h2d = sum(s.h2d_bytes() for s in shapes)
+    d2h = sum(s.d2h_bytes() for s in shapes)
+
+    # ---- roofline of the dominant kernel (prefill_kernel, the only kernel of the step)
+    peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flops_step * args.steps / (sum(sum(v) for v in per_shape_ms.values()) / 1e3) / 1e12
+    big = HEADLINE[-1].name
+    traffic = measured_traffic(big)
+    roofline = {"bound": "tensor", "kernel": "prefill_kernel<128,4>", "achieved": round(achieved, 1),
+                "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
+                "peak_kind": f"{peaks_kind} bf16 dense (burst)", "traffic": traffic,
+                "traffic_workload": big}
+
+    breakdown = {}
+    for s in shapes:
+        ts = per_shape_ms[s.w.name]
+        med = statistics.median(ts)
+        breakdown[s.w.name] = {"ms": round(med, 4), "tflops": round(s.w.flops() / med / 1e9, 1),
+                               "frac": round(s.w.flops() / med / 1e9 / peak_tf, 4)}
+    del shapes
+    if not args.no_breakdown:
+        breakdown.update(measure_breakdown(flush, peak_tf, float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
+                                           rank))
+    sdpa.check_device_error()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, cores, desc, _ = CpuOracleSample(HEADLINE[-1]).sample(target_s=12.0)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "wall_ms_per_step": round(wall * 1e3 / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded randn N(0,1), rounded to bf16)",
+            "config": {"workload": "prefill non-causal d=128 H=16 seq {512,1024,2048,4096} B=16384/seq "
+                                   "(one call per shape per step)",
+                       "global_batch_tokens": 16384 * 4 * world, "seq_len": [w.Sq for w in HEADLINE],
+                       "heads": 16, "head_dim": 128, "causal": False, "parallelism": f"replicas x{world}",
+                       "l2": "flushed (256 MiB write) before every call"},
+            "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": len(HEADLINE) * args.steps,
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "clocks": clocks.summary(),
+            "breakdown": breakdown,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def measure_breakdown(flush, peak_tf, hbm_gbs, rank, reps: int = 10):
+    out = {}
+    for w in inputs.PREFILL_CAUSAL + [inputs.GQA_LONG]:
+        s = GpuPrefill(w, rank)
+        ms = statistics.median(timed_calls([s.run], flush, reps, 3)[0])
+        tf = w.flops() / ms / 1e9
+        out[w.name] = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac": round(tf / peak_tf, 4)}
+        del s
+    for w in inputs.DECODE:
+        s = GpuDecode(w, rank)
+        ms = statistics.median(timed_calls([s.run], flush, reps * 3, 5)[0])
+        gbs = w.decode_bytes() / ms / 1e6
+        out[w.name] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4),
+                       "splits": int(s.ws.numel() // (w.B * w.Hq * w.Sq * (w.d + 2) * 4)),
+                       "launches_per_call": 2}
+        del s
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 oracle as it stands, on the host cores,
+    on a bounded sample of the headline workload (rank 0 only)."""
+    if rank != 0:
+        return
+    w = HEADLINE[-1]
+    sampler = CpuOracleSample(w)
+    vals = []
+    for i in range(args.warmup + args.steps):
+        tf, cores, desc, dt = sampler.sample(target_s=max(1.0, 60.0 / max(1, args.warmup + args.steps)))
+        if i >= args.warmup:
+            vals.append((tf, dt))
+    tf = statistics.median(v for v, _ in vals)
+    line = {"impl": "reference", "metric": METRIC, "value": round(tf, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * statistics.median(dt for _, dt in vals), 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded randn N(0,1), rounded to bf16)",
+            "config": {"workload": f"{w.name}: row sample of the prefill non-causal d=128 H=16 workload"},
+            "cpu_baseline": {"value": round(tf, 6), "unit": "TFLOP/s", "cores": os.cpu_count() or 1,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(tf, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,140 @@
+/*
+ * sdpa_b200.h -- C ABI of libsdpa_b200.so: fused scaled-dot-product attention
+ * forward (prefill) and split-KV decode for NVIDIA B200 (sm_100a).
+ *
+ * The operation, for every batch b, query head hq and query row i, with
+ * hk = hq / (Hq / Hkv):
+ *     x_ij  = scale * sum_c q[b,hq,i,c] * k[b,hk,j,c]           (matmul, scale)
+ *     x_ij  = -inf where key j is masked for row i               (masked_fill)
+ *     p_ij  = exp(x_ij - max_j x_ij) / sum_j exp(x_ij - max_j x_ij)   (softmax)
+ *     o[b,hq,i,:] = sum_j p_ij v[b,hk,j,:]                       (matmul)
+ *     lse[b,hq,i] = max_j x_ij + ln sum_j exp(x_ij - max_j x_ij)
+ * -- the five naive steps of "PyTorch attention profiling: Flash, cuDNN, Math
+ * backends" (section 1), computed the FlashAttention-2 way ("FlashAttention-2"
+ * notes, algorithm overview: per query block, online max/sum over key blocks,
+ * one final division).  A row with no visible key gets o = 0 and
+ * lse = -inf (the no-NaN intent of that page's "_safe_softmax").
+ *
+ * Masks (`causal`):
+ *   ATTN_CAUSAL_NONE          every key visible
+ *   ATTN_CAUSAL_TOP_LEFT      key j visible to row i iff j <= i
+ *   ATTN_CAUSAL_BOTTOM_RIGHT  key j visible to row i iff j <= i + Sk - Sq
+ *                             (query rows sit at the end of the keys)
+ * Scale: scale == 0 selects 1/sqrt(d) (the default-alpha rule of the
+ * onnxruntime WebGPU decode page, section 2); otherwise it must be finite and
+ * > 0.
+ *
+ * Layout and types: every tensor is contiguous, row-major.
+ *   q, o          [B, Hq,  Sq, d]  bf16
+ *   k, v          [B, Hkv, Sk, d]  bf16
+ *   lse           [B, Hq,  Sq]     fp32 (may be NULL)
+ * d must be 64 or 128; Hq must be a multiple of Hkv (GQA: query head hq
+ * reads KV head hq / (Hq/Hkv), no expansion).  q, k, v, o must be 16-byte
+ * aligned device pointers; lse 4-byte aligned.
+ *
+ * Ownership: the caller allocates and owns every buffer, including the
+ * decode workspace.  The library allocates no device memory per call (one
+ * 4-byte device error word per process, and nothing else) and keeps no
+ * per-call search.  Calls are asynchronous on `stream` (a cudaStream_t
+ * passed as void*; NULL = legacy default stream) and never synchronize.
+ *
+ * Errors: argument errors are detected on the host before anything is
+ * launched and returned synchronously; ATTN_ERR_CUDA is returned when a
+ * CUDA runtime call fails (launch, attribute, tensor-map encoding).  Every
+ * wait inside the kernels is bounded (1 s); a wait that gives up records a
+ * bit in the device error word and the kernel exits without trapping;
+ * attn_check_device_error() reports it as ATTN_ERR_DEVICE_TIMEOUT.
+ * No function ever aborts the process.
+ */
+#ifndef SDPA_B200_H
+#define SDPA_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_NULL = 1,           /* a required pointer is NULL */
+  ATTN_ERR_SHAPE = 2,          /* negative size, or a size beyond the supported range */
+  ATTN_ERR_GQA = 3,            /* Hq is not a multiple of Hkv */
+  ATTN_ERR_HEADDIM = 4,        /* d is not 64 or 128 */
+  ATTN_ERR_ALIGN = 5,          /* a pointer is not 16-byte (lse: 4-byte) aligned */
+  ATTN_ERR_CAUSAL = 6,         /* unknown causal mode, or a mode the entry point lacks */
+  ATTN_ERR_WORKSPACE = 7,      /* decode workspace NULL, misaligned or too small */
+  ATTN_ERR_CUDA = 8,           /* a CUDA runtime call failed */
+  ATTN_ERR_DEVICE_TIMEOUT = 9, /* a bounded wait inside a kernel gave up */
+  ATTN_ERR_ARCH = 10,          /* the current device is not compute capability 10.0 */
+  ATTN_ERR_SCALE = 11          /* scale is negative, NaN or infinite */
+} attn_status_t;
+
+enum { ATTN_CAUSAL_NONE = 0, ATTN_CAUSAL_TOP_LEFT = 1, ATTN_CAUSAL_BOTTOM_RIGHT = 2 };
+
+/*
+ * Prefill / general forward.  Computes o (and lse when non-NULL) for any
+ * Sq >= 0, Sk >= 0.  Work items are (b, hq, block of 256 query rows); each
+ * visits only the key blocks its causal mask leaves visible ("FlashAttention-2"
+ * notes, causal masking and sequence-length parallelism).
+ */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                       int Sq, int Sk, int d, float scale, int causal, void* stream);
+
+/*
+ * Number of KV splits attn_decode_splitkv uses for this shape when called
+ * with num_splits = 0 (picked to fill the device's SMs).  Needs the current
+ * device's SM count; without a device it assumes 148.  Returns 0 for an
+ * invalid shape.
+ */
+int attn_decode_num_splits(int B, int Hq, int Hkv, int Sq, int Sk, int d);
+
+/*
+ * Bytes of workspace attn_decode_splitkv needs: fp32 partial outputs
+ * [B*Hq*Sq][splits][d] plus fp32 (max, sum) pairs [B*Hq*Sq][splits], with
+ * `splits` the effective split count for num_splits (0 = automatic).
+ * Returns 0 for an invalid shape.
+ */
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int d, int num_splits);
+
+/*
+ * Split-KV decode ("[onnxruntime] WebGPU FlashAttention: kernel fusion and
+ * variable sequence length", section 1): the keys of each (b, kv head) are
+ * cut into splits of whole 64-key tiles; one kernel computes, per split, the
+ * locally normalised partial output and its (local max, local sum); a
+ * second kernel combines the splits by log-sum-exp rescaling into o and lse.
+ * The result equals attn_fwd on the same inputs up to rounding.
+ *   k_cache, v_cache  [B, Hkv, Sk, d] bf16 (every position valid)
+ *   causal            ATTN_CAUSAL_NONE or ATTN_CAUSAL_BOTTOM_RIGHT (rows at
+ *                     the end of the cache) or ATTN_CAUSAL_TOP_LEFT
+ *   num_splits        0 = automatic; otherwise the requested count, rounded
+ *                     to whole 64-key tiles (never more than ceil(Sk/64))
+ *   workspace         device buffer of at least
+ *                     attn_decode_workspace_size(...) bytes, 16-byte aligned;
+ *                     owned by the caller, overwritten by the call.
+ * Each CTA serves the G*Sq <= 16 query rows of one KV head at a time (G =
+ * Hq/Hkv); larger G*Sq is handled in groups of 16 rows.
+ */
+attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                                  int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale, int causal,
+                                  int num_splits, void* workspace, size_t workspace_bytes, void* stream);
+
+/* A static, human-readable name for a status code. */
+const char* attn_status_string(attn_status_t status);
+
+/*
+ * Synchronizes `stream`, then reads and clears the device error word.
+ * Returns ATTN_ERR_DEVICE_TIMEOUT if a kernel gave up on a bounded wait since
+ * the last check, ATTN_ERR_CUDA if the synchronization itself failed, else
+ * ATTN_OK.
+ */
+attn_status_t attn_check_device_error(void* stream);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDPA_B200_H */

@@ -1,0 +1,393 @@
+// decode.cuh -- split-KV decode attention and the log-sum-exp combine.
+//
+// The method is the fused decode of "[onnxruntime] WebGPU FlashAttention:
+// kernel fusion and variable sequence length", section 1: one kernel computes,
+// per KV split, Q K^T, the causal mask, a local softmax and the product with
+// V, and writes a LOCALLY normalised partial output plus (local max, local
+// sum) metadata; a second, reduce kernel rescales the partials with that
+// metadata so the result equals full softmax(Q K^T) V.  Section 2 of the
+// same page amortises one K/V load over several query rows (m_tile); here a
+// CTA serves every query row that shares its KV head (G = Hq/Hkv heads times
+// Sq rows, up to 16 per CTA).
+//
+// B200 mapping (this file's own design):
+//   * grid = (row group, split, batch*kv_head); 4 consumer warps + 1 TMA
+//     producer warp; K/V tiles of 64 keys stream through an NSTAGE-deep ring
+//     of 128-byte-swizzled shared-memory tiles.
+//   * The work per byte is tiny (<= 16 query rows), so the contraction runs on
+//     warp-level mma.sync m16n8k16 (bf16, fp32 accumulate): the kernel is
+//     bound by HBM bandwidth, not by the tensor pipe.  Each warp owns 16 keys
+//     of every tile and its own running (m, l, O); the four warps merge once
+//     through shared memory at the end.
+//   * The combine kernel is one warp per output row with 16-byte coalesced
+//     loads of the fp32 partials.
+#pragma once
+#include "ptx.cuh"
+
+namespace sdpa {
+
+struct DecodeParams {
+  CUtensorMap tm_k;       // [B*Hkv][Sk][d] bf16, box {64, 64, 1}, 128-byte swizzle
+  CUtensorMap tm_v;       // [B*Hkv][Sk][d]
+  const uint16_t* q;      // [B, Hq, Sq, d] bf16 bits
+  float* part_o;          // [B*Hq*Sq][nsplit][d]  locally normalised partial outputs
+  float2* part_ml;        // [B*Hq*Sq][nsplit]     (local max of scale*q.k, local sum)
+  int B, Hq, Hkv, Sq, Sk, group;
+  int causal, causal_offset;  // key j visible to row i iff j <= i + causal_offset (if causal)
+  int nsplit;             // splits per (batch, kv head)
+  int tiles_per_split;    // 64-key tiles per split
+  int row_groups;         // ceil(group*Sq / 16)
+  float scale, scale_log2;
+};
+
+constexpr int kDecKeys = 64;          // keys per tile
+constexpr int kDecRows = 16;          // query rows per CTA (mma M)
+constexpr int kDecThreads = 160;      // 4 consumer warps + 1 producer warp
+constexpr int kDecProducerWarp = 4;
+
+template <int D, int NSTAGE>
+struct DecodeCfg {
+  static constexpr int kBoxBytes = kDecKeys * 128;         // one 64-key x 64-col swizzle block
+  static constexpr int kHalfBytes = kBoxBytes * (D / 64);  // K or V tile
+  static constexpr int kStageBytes = 2 * kHalfBytes;
+  static constexpr int kMergeBytes = 4 * kDecRows * D * 4 + 2 * 4 * kDecRows * 4;
+  static constexpr int kRingBytes = NSTAGE * kStageBytes > kMergeBytes ? NSTAGE * kStageBytes : kMergeBytes;
+  static constexpr int kSmemBytes = kRingBytes + 2 * NSTAGE * 8 + 16 + 1024;
+};
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                                  uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D(16x8, f32) += A(16x16, bf16, row) * B(16x8, bf16, col)
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Byte offset of element (key r, column c) inside a 128-byte-swizzled tile of
+// 64-column blocks with `rows` rows per block (16-byte chunk granularity).
+__device__ __forceinline__ uint32_t sw128_off(int r, int c, int block_bytes) {
+  return (c >> 6) * block_bytes + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1);
+}
+
+template <int D, int NSTAGE>
+__global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_constant__ DecodeParams p) {
+  using Cfg = DecodeCfg<D, NSTAGE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t ring = smem_u32(smem);
+  const uint32_t bar0 = ring + Cfg::kRingBytes;
+  auto full = [&](int s) { return bar0 + 8u * s; };             // [NSTAGE] stage filled
+  auto empty = [&](int s) { return bar0 + 8u * (NSTAGE + s); }; // [NSTAGE] stage released
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kRingBytes + 16 * NSTAGE);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rg = static_cast<int>(blockIdx.x) % p.row_groups;
+  const int split = (static_cast<int>(blockIdx.x) / p.row_groups) % p.nsplit;
+  const int bhkv = static_cast<int>(blockIdx.x) / (p.row_groups * p.nsplit);
+  const int b = bhkv / p.Hkv;
+  const int hkv = bhkv - b * p.Hkv;
+  const int rows_total = p.group * p.Sq;  // query rows sharing this KV head
+  const int total_tiles = (p.Sk + kDecKeys - 1) / kDecKeys;
+  const int tile_begin = split * p.tiles_per_split;
+  const int tile_end = min(total_tiles, tile_begin + p.tiles_per_split);
+  const int ntiles = max(0, tile_end - tile_begin);
+  // first flattened (b*Hq + hq)*Sq + i row of this KV head
+  const int64_t row_base = (static_cast<int64_t>(b) * p.Hq + static_cast<int64_t>(hkv) * p.group) * p.Sq;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 4);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kDecProducerWarp) {
+    if (lane == 0 && ntiles > 0) {
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      int issued = 0;
+      for (int it = 0; it < ntiles; ++it) {
+        const int st = it % NSTAGE;
+        if (!mbar_wait(empty(st), ((it / NSTAGE) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(full(st), Cfg::kStageBytes);
+        const uint32_t sk = ring + st * Cfg::kStageBytes;
+        const uint32_t sv = sk + Cfg::kHalfBytes;
+        const int key0 = (tile_begin + it) * kDecKeys;
+#pragma unroll
+        for (int blk = 0; blk < D / 64; ++blk) {
+          tma_load_3d(sk + blk * Cfg::kBoxBytes, &p.tm_k, blk * 64, key0, bhkv, full(st));
+          tma_load_3d(sv + blk * Cfg::kBoxBytes, &p.tm_v, blk * 64, key0, bhkv, full(st));
+        }
+        ++issued;
+      }
+      for (int it = max(0, issued - NSTAGE); it < issued; ++it) mbar_wait_drain(full(it % NSTAGE), (it / NSTAGE) & 1);
+    }
+    __syncwarp();
+    named_bar_sync(1, kDecThreads);  // matches the consumers' barrier before the merge
+    named_bar_sync(1, kDecThreads);  // matches the consumers' barrier after the merge writes
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers
+  const float c = p.scale_log2;
+  const int qr = lane >> 2;        // fragment row (and row + 8)
+  const int qc = (lane & 3) * 2;   // fragment column pair
+  // Query rows of this CTA: r in [0,16) -> local row rg*16 + r of this KV head.
+  uint32_t qf[D / 16][4];
+  {
+    const int r_lo = rg * kDecRows + qr;
+    const int r_hi = r_lo + 8;
+    const uint32_t* q_lo = reinterpret_cast<const uint32_t*>(p.q + (row_base + r_lo) * D);
+    const uint32_t* q_hi = reinterpret_cast<const uint32_t*>(p.q + (row_base + r_hi) * D);
+    const bool v_lo = r_lo < rows_total, v_hi = r_hi < rows_total;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      qf[ks][0] = v_lo ? q_lo[(ks * 16 + qc) >> 1] : 0u;
+      qf[ks][1] = v_hi ? q_hi[(ks * 16 + qc) >> 1] : 0u;
+      qf[ks][2] = v_lo ? q_lo[(ks * 16 + 8 + qc) >> 1] : 0u;
+      qf[ks][3] = v_hi ? q_hi[(ks * 16 + 8 + qc) >> 1] : 0u;
+    }
+  }
+  // causal limit per fragment row: the last key each row may see
+  int lim[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int lr = rg * kDecRows + qr + 8 * h;  // local row = g*Sq + i
+    const int i = lr % p.Sq;
+    lim[h] = p.causal ? min(p.Sk - 1, i + p.causal_offset) : p.Sk - 1;
+  }
+
+  float o[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m[2] = {-INFINITY, -INFINITY};
+  float l[2] = {0.f, 0.f};
+  bool ok = true;
+
+  for (int it = 0; it < ntiles; ++it) {
+    const int st = it % NSTAGE;
+    if (!mbar_wait(full(st), (it / NSTAGE) & 1, abort_flag)) {
+      ok = false;
+      break;
+    }
+    const uint32_t sk = ring + st * Cfg::kStageBytes;
+    const uint32_t sv = sk + Cfg::kHalfBytes;
+    const int kb = warp * 16;  // this warp's 16 keys inside the tile
+    // ---- S = Q K^T for 16 rows x 16 keys
+    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    {
+      const int mi = lane >> 3;
+      const int key = kb + (mi >> 1) * 8 + (lane & 7);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4(sk + sw128_off(key, ks * 16 + (mi & 1) * 8, Cfg::kBoxBytes), b0, b1, b2, b3);
+        mma_bf16_16816(sc[0], qf[ks], b0, b1);
+        mma_bf16_16816(sc[1], qf[ks], b2, b3);
+      }
+    }
+    // ---- mask, online softmax (rows qr and qr+8 of this thread)
+    const int key0 = (tile_begin + it) * kDecKeys + kb;
+    if (key0 + 15 > min(lim[0], lim[1])) {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = key0 + nt * 8 + qc + (e & 1);
+          if (key > lim[e >> 1]) sc[nt][e] = -INFINITY;
+        }
+    }
+    float alpha[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float mx = fmaxf(fmaxf(sc[0][2 * h], sc[0][2 * h + 1]), fmaxf(sc[1][2 * h], sc[1][2 * h + 1]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = fmaxf(m[h], mx);
+      alpha[h] = (m[h] == -INFINITY) ? 0.f : ex2_approx((m[h] - m_new) * c);
+      m[h] = m_new;
+    }
+    uint32_t pa[4];
+    {
+      const float mc0 = (m[0] == -INFINITY) ? 0.f : m[0] * c;
+      const float mc1 = (m[1] == -INFINITY) ? 0.f : m[1] * c;
+      float p00 = ex2_approx(fmaf(sc[0][0], c, -mc0)), p01 = ex2_approx(fmaf(sc[0][1], c, -mc0));
+      float p02 = ex2_approx(fmaf(sc[0][2], c, -mc1)), p03 = ex2_approx(fmaf(sc[0][3], c, -mc1));
+      float p10 = ex2_approx(fmaf(sc[1][0], c, -mc0)), p11 = ex2_approx(fmaf(sc[1][1], c, -mc0));
+      float p12 = ex2_approx(fmaf(sc[1][2], c, -mc1)), p13 = ex2_approx(fmaf(sc[1][3], c, -mc1));
+      l[0] = l[0] * alpha[0] + (p00 + p01 + p10 + p11);
+      l[1] = l[1] * alpha[1] + (p02 + p03 + p12 + p13);
+      pa[0] = pack_bf16x2(p00, p01);
+      pa[1] = pack_bf16x2(p02, p03);
+      pa[2] = pack_bf16x2(p10, p11);
+      pa[3] = pack_bf16x2(p12, p13);
+    }
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      o[n][0] *= alpha[0];
+      o[n][1] *= alpha[0];
+      o[n][2] *= alpha[1];
+      o[n][3] *= alpha[1];
+    }
+    // ---- O += P V  (V^T fragments through ldmatrix.trans)
+    {
+      const int mi = lane >> 3;
+      const int key = kb + (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+      for (int n = 0; n < D / 8; n += 2) {
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4_trans(sv + sw128_off(key, (n + (mi >> 1)) * 8, Cfg::kBoxBytes), b0, b1, b2, b3);
+        mma_bf16_16816(o[n], pa, b0, b1);
+        mma_bf16_16816(o[n + 1], pa, b2, b3);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty(st));
+  }
+
+  // ---- merge the four warps' (m, l, O) through shared memory
+  // (quad-reduce l first: each thread summed only its own columns)
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 1);
+    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 2);
+  }
+  named_bar_sync(1, kDecThreads);  // every warp is past the ring: reuse it for the merge
+  float* s_o = reinterpret_cast<float*>(smem);          // [4][16][D]
+  float* s_m = s_o + 4 * kDecRows * D;                   // [4][16]
+  float* s_l = s_m + 4 * kDecRows;                       // [4][16]
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) {
+    *reinterpret_cast<float2*>(&s_o[(warp * kDecRows + qr) * D + n * 8 + qc]) = make_float2(o[n][0], o[n][1]);
+    *reinterpret_cast<float2*>(&s_o[(warp * kDecRows + qr + 8) * D + n * 8 + qc]) = make_float2(o[n][2], o[n][3]);
+  }
+  if ((lane & 3) == 0) {
+    s_m[warp * kDecRows + qr] = m[0];
+    s_m[warp * kDecRows + qr + 8] = m[1];
+    s_l[warp * kDecRows + qr] = l[0];
+    s_l[warp * kDecRows + qr + 8] = l[1];
+  }
+  named_bar_sync(1, kDecThreads);
+  if (!ok) return;
+  // thread t: row t/8, 16 (D=128) or 8 (D=64) consecutive columns
+  {
+    const int r = threadIdx.x >> 3;
+    const int lr = rg * kDecRows + r;
+    if (lr < rows_total) {
+      constexpr int kCols = D / 8;
+      const int c0 = (threadIdx.x & 7) * kCols;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 4; ++w)
+        if (s_l[w * kDecRows + r] > 0.f) M = fmaxf(M, s_m[w * kDecRows + r]);
+      float wt[4];
+      float L = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float lw = s_l[w * kDecRows + r];
+        wt[w] = (lw > 0.f) ? ex2_approx((s_m[w * kDecRows + r] - M) * c) : 0.f;
+        L += wt[w] * lw;
+      }
+      const float inv = (L > 0.f) ? 1.f / L : 0.f;
+      const int64_t row = row_base + lr;
+      float* dst = p.part_o + (row * p.nsplit + split) * D + c0;
+#pragma unroll
+      for (int cc = 0; cc < kCols; cc += 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float4 v = *reinterpret_cast<const float4*>(&s_o[(w * kDecRows + r) * D + c0 + cc]);
+          acc.x += wt[w] * v.x;
+          acc.y += wt[w] * v.y;
+          acc.z += wt[w] * v.z;
+          acc.w += wt[w] * v.w;
+        }
+        acc.x *= inv;
+        acc.y *= inv;
+        acc.z *= inv;
+        acc.w *= inv;
+        *reinterpret_cast<float4*>(dst + cc) = acc;
+      }
+      if ((threadIdx.x & 7) == 0)
+        p.part_ml[row * p.nsplit + split] = make_float2(L > 0.f ? M * p.scale : -INFINITY, L);
+    }
+  }
+}
+
+// One warp per output row: O = sum_s w_s O_s / sum_s w_s with
+// w_s = l_s exp(m_s - M), M = max_s m_s; LSE = M + ln(sum_s w_s).  A split
+// with l_s = 0 saw no visible key and gets weight 0; a row whose splits are
+// all empty gets O = 0 and LSE = -inf.
+template <int D>
+__global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ part_o,
+                                                             const float2* __restrict__ part_ml,
+                                                             uint16_t* __restrict__ out, float* __restrict__ lse,
+                                                             int64_t rows, int nsplit) {
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  constexpr int kPer = D / 32;  // floats per lane: 4 (one 16-byte load) or 2
+  constexpr float kLog2e = 1.4426950408889634f;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const float2* ml = part_ml + row * nsplit;
+  float M = -INFINITY;
+  for (int s = lane; s < nsplit; s += 32) {
+    const float2 v = ml[s];
+    if (v.y > 0.f) M = fmaxf(M, v.x);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  float W = 0.f;
+  if (M != -INFINITY) {
+    const float* po = part_o + row * nsplit * D + lane * kPer;
+    for (int s = 0; s < nsplit; ++s) {
+      const float2 v = ml[s];
+      const float w = (v.y > 0.f) ? v.y * ex2_approx((v.x - M) * kLog2e) : 0.f;
+      W += w;
+      if constexpr (kPer == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(po + static_cast<int64_t>(s) * D);
+        acc[0] += w * x.x;
+        acc[1] += w * x.y;
+        acc[2] += w * x.z;
+        acc[3] += w * x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2*>(po + static_cast<int64_t>(s) * D);
+        acc[0] += w * x.x;
+        acc[1] += w * x.y;
+      }
+    }
+  }
+  const float inv = (W > 0.f) ? 1.f / W : 0.f;
+  uint16_t* dst = out + row * D + lane * kPer;
+  if constexpr (kPer == 4) {
+    *reinterpret_cast<uint2*>(dst) =
+        make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  }
+  if (lane == 0 && lse != nullptr)
+    lse[row] = (W > 0.f) ? M + lg2_approx(W) * 0.69314718055994531f : -INFINITY;
+}
+
+}  // namespace sdpa

@@ -1,0 +1,431 @@
+// prefill.cuh -- fused attention forward (prefill) for sm_100a.
+//
+// O = softmax(scale * Q K^T + causal mask) V, with LSE, bf16 in / bf16 out,
+// fp32 accumulation.  The loop structure is the FlashAttention-2 forward
+// ("FlashAttention-2" notes, algorithm overview): each query block keeps a
+// running row max m and row sum l, walks the key/value blocks, and divides by
+// l once at the end; fully masked causal blocks are never visited (same
+// notes, causal masking); the parallel work items are (batch, head, query
+// block) (same notes, improvement 2: sequence-length parallelism).
+//
+// B200 mapping (this file's own design, not the pages'):
+//   * one CTA = two 128-row query tiles of one (batch, head) sharing every
+//     K/V tile it loads; 12 warps (3 warpgroups):
+//       warps 0-3  softmax group 0 (one thread per row of query tile 0)
+//       warps 4-7  softmax group 1 (query tile 1)
+//       warp  8    MMA issuer (one elected thread) + TMEM owner
+//       warp  9    TMA producer (one elected thread)
+//       warps 10-11 idle
+//     The block launches at kLaunchRegs registers per thread; warpgroup 2
+//     gives registers back (kCtrlRegs) so the softmax warpgroups can hold a
+//     full 128-column S row in registers (kSoftmaxRegs).  The split adds up
+//     to exactly the launch allocation: 256*kSoftmaxRegs + 128*kCtrlRegs ==
+//     384*kLaunchRegs.
+//   * TMEM (512 columns): S0 | S1 | O0 | O1.  P (bf16) is written over the
+//     first half of its own S columns and consumed from TMEM by the P.V MMA.
+//   * K/V tiles stream through an NS-slot shared-memory ring (K_j, V_j in
+//     consecutive slots), 128-byte swizzled, filled by TMA, released by
+//     tcgen05.commit when the MMAs reading them are done.
+//   * The two query tiles ping-pong: while softmax group 0 works on S0(j)
+//     the tensor core runs P1.V and S1(j+1), and vice versa.
+//   * Rescaling of O is skipped unless the running max grows by more than
+//     2^8 in the exp2 domain (exact: the final O/l and LSE use the same m).
+#pragma once
+#include <climits>
+
+#include "ptx.cuh"
+
+namespace sdpa {
+
+struct PrefillParams {
+  CUtensorMap tm_q;  // [B*Hq][Sq][d] bf16, box {64, 128, 1}, 128-byte swizzle
+  CUtensorMap tm_k;  // [B*Hkv][Sk][d]
+  CUtensorMap tm_v;  // [B*Hkv][Sk][d]
+  CUtensorMap tm_o;  // [B*Hq][Sq][d]
+  float* lse;        // [B*Hq*Sq] or nullptr
+  int B, Hq, Hkv, Sq, Sk;
+  int group;          // Hq / Hkv
+  int causal;         // 0 none, 1 top-left, 2 bottom-right
+  int causal_offset;  // key j visible to row i iff j <= i + causal_offset
+  int num_units;      // ceil(Sq / 256): CTAs per (batch, head)
+  int lpt;            // 1: launch the heaviest units first (causal)
+  float scale;        // softmax scale on q.k
+  float scale_log2;   // scale * log2(e)
+};
+
+constexpr int kBlockM = 128;  // query rows per tile
+constexpr int kBlockN = 128;  // keys per tile
+constexpr int kPrefillThreads = 384;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr int kLaunchRegs = 168;   // 3 warps per SM sub-partition: 3*32*168 <= 16384
+constexpr int kSoftmaxRegs = 224;
+constexpr int kCtrlRegs = 56;
+static_assert(256 * kSoftmaxRegs + 128 * kCtrlRegs == kPrefillThreads * kLaunchRegs,
+              "register split must equal the launch allocation");
+constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest P kept unrescaled
+
+template <int D, int NS>
+struct PrefillCfg {
+  static constexpr int kTileBytes = kBlockM * D * 2;  // one Q, K or V tile (bf16)
+  static constexpr int kBlocks = D / 64;               // 64-column swizzle blocks per tile
+  static constexpr int kBlockBytes = kBlockM * 128;    // 16 KB per swizzle block
+  static constexpr int kNumBars = 2 + 2 * NS + 2 + 2 + 2 + 1;
+  static constexpr int kSmemBytes = (2 + NS) * kTileBytes + kNumBars * 8 + 16 + 1024;
+};
+
+// Number of key tiles the query tile starting at row0 must visit.
+__device__ __forceinline__ int kv_tiles_for(const PrefillParams& p, int row0) {
+  if (row0 >= p.Sq || p.Sk <= 0) return 0;
+  int last_key = p.Sk - 1;
+  if (p.causal) {
+    const int last_row = min(row0 + kBlockM - 1, p.Sq - 1);
+    last_key = min(last_key, last_row + p.causal_offset);
+  }
+  if (last_key < 0) return 0;
+  return last_key / kBlockN + 1;
+}
+
+template <int D, int NS>
+__global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
+  using Cfg = PrefillCfg<D, NS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // Shared-memory map (32-bit shared addresses):
+  //   sQ   2 query tiles, sKV NS key/value slots, then the barriers.
+  const uint32_t sQ = smem_u32(smem);
+  const uint32_t sKV = sQ + 2 * Cfg::kTileBytes;
+  const uint32_t bar0 = sKV + NS * Cfg::kTileBytes;
+  auto q_full = [&](int t) { return bar0 + 8u * t; };                 // [2] Q_t landed
+  auto kv_full = [&](int s) { return bar0 + 8u * (2 + s); };          // [NS] slot filled
+  auto kv_empty = [&](int s) { return bar0 + 8u * (2 + NS + s); };    // [NS] slot released
+  auto s_full = [&](int t) { return bar0 + 8u * (2 + 2 * NS + t); };  // [2] S_t(j) ready (P_t.V(j-1) done)
+  auto p_full = [&](int t) { return bar0 + 8u * (4 + 2 * NS + t); };  // [2] P_t(j) written (O_t rescaled)
+  auto o_full = [&](int t) { return bar0 + 8u * (6 + 2 * NS + t); };  // [2] last P_t.V done
+  const uint32_t drain = bar0 + 8u * (8 + 2 * NS);                    // every MMA done
+  uint8_t* bar_ptr = smem + 2 * Cfg::kTileBytes + NS * Cfg::kTileBytes;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * Cfg::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: (batch*head, pair of query tiles)
+  const int BH = p.B * p.Hq;
+  int bh, unit;
+  if (p.lpt) {
+    unit = p.num_units - 1 - static_cast<int>(blockIdx.x) / BH;
+    bh = static_cast<int>(blockIdx.x) % BH;
+  } else {
+    unit = static_cast<int>(blockIdx.x) % p.num_units;
+    bh = static_cast<int>(blockIdx.x) / p.num_units;
+  }
+  const int b = bh / p.Hq;
+  const int hq = bh - b * p.Hq;
+  const int bhkv = b * p.Hkv + hq / p.group;
+  const int row0_0 = unit * 2 * kBlockM;
+  const int row0_1 = row0_0 + kBlockM;
+  const int n0 = kv_tiles_for(p, row0_0);
+  const int n1 = kv_tiles_for(p, row0_1);
+  const int n_max = max(n0, n1);
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(q_full(t), 1);
+      mbar_init(s_full(t), 1);
+      mbar_init(p_full(t), 4);  // one arrive per softmax warp
+      mbar_init(o_full(t), 1);
+    }
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+    // Warpgroup 2 (control): every warp runs the same setmaxnreg first.
+    regs_decrease<kCtrlRegs>();
+    if (warp == kLoadWarp) {
+      // ------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        tma_prefetch_desc(&p.tm_q);
+        tma_prefetch_desc(&p.tm_k);
+        tma_prefetch_desc(&p.tm_v);
+        tma_prefetch_desc(&p.tm_o);
+        if (n0 > 0) {
+          mbar_arrive_expect_tx(q_full(0), Cfg::kTileBytes);
+          for (int blk = 0; blk < Cfg::kBlocks; ++blk)
+            tma_load_3d(sQ + blk * Cfg::kBlockBytes, &p.tm_q, blk * 64, row0_0, bh, q_full(0));
+        }
+        if (n1 > 0) {
+          mbar_arrive_expect_tx(q_full(1), Cfg::kTileBytes);
+          for (int blk = 0; blk < Cfg::kBlocks; ++blk)
+            tma_load_3d(sQ + Cfg::kTileBytes + blk * Cfg::kBlockBytes, &p.tm_q, blk * 64, row0_1, bh, q_full(1));
+        }
+        int issued = 0;
+        const int total = 2 * n_max;  // K_0, V_0, K_1, V_1, ...
+#pragma unroll 1
+        for (int it = 0; it < total; ++it) {
+          const int slot = it % NS;
+          if (!mbar_wait(kv_empty(slot), ((it / NS) & 1) ^ 1, abort_flag)) break;
+          mbar_arrive_expect_tx(kv_full(slot), Cfg::kTileBytes);
+          const CUtensorMap* tm = (it & 1) ? &p.tm_v : &p.tm_k;
+          const uint32_t dst = sKV + slot * Cfg::kTileBytes;
+          for (int blk = 0; blk < Cfg::kBlocks; ++blk)
+            tma_load_3d(dst + blk * Cfg::kBlockBytes, tm, blk * 64, (it >> 1) * kBlockN, bhkv, kv_full(slot));
+          ++issued;
+        }
+        // Copies still in flight must land before the CTA may exit.
+        if (n0 > 0) mbar_wait_drain(q_full(0), 0);
+        if (n1 > 0) mbar_wait_drain(q_full(1), 0);
+        for (int it = max(0, issued - NS); it < issued; ++it) mbar_wait_drain(kv_full(it % NS), (it / NS) & 1);
+      }
+      __syncwarp();
+    } else if (warp == kMmaWarp) {
+      // --------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t kIdS = idesc_bf16_f32(kBlockM, kBlockN, false);
+        constexpr uint32_t kIdPV = idesc_bf16_f32(kBlockM, D, true);
+        constexpr uint32_t kHiK = sdesc_hi(1024);  // K-major: 8-row groups 1024 B apart
+        constexpr uint32_t kHiV = sdesc_hi(1024);  // MN-major: 8-key groups 1024 B apart
+        bool ok = true;
+        // S_t = Q_t K^T over D in steps of 16 (32 bytes inside a 128-byte swizzle row,
+        // next 64-column block 16 KB further).
+        auto issue_s = [&](int t, int slot) {
+          const uint32_t qa = sQ + t * Cfg::kTileBytes;
+          const uint32_t ka = sKV + slot * Cfg::kTileBytes;
+#pragma unroll 1
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * Cfg::kBlockBytes + (kk & 3) * 32;
+            const uint64_t da = (static_cast<uint64_t>(kHiK) << 32) | sdesc_lo(qa + off, 16);
+            const uint64_t db = (static_cast<uint64_t>(kHiK) << 32) | sdesc_lo(ka + off, 16);
+            mma_ss(tmem + t * kBlockN, da, db, kIdS, kk > 0 ? 1u : 0u);
+          }
+        };
+        // O_t (+)= P_t V over the 128 keys in steps of 16 (8 TMEM columns of
+        // packed bf16 P; 16 rows of V = 2048 bytes).  V is MN-major: its two
+        // 64-column blocks are 16 KB apart (leading byte offset).
+        auto issue_pv = [&](int t, int slot, bool acc) {
+          const uint32_t va = sKV + slot * Cfg::kTileBytes;
+#pragma unroll 1
+          for (int kk = 0; kk < kBlockN / 16; ++kk) {
+            const uint64_t db = (static_cast<uint64_t>(kHiV) << 32) | sdesc_lo(va + kk * 2048, Cfg::kBlockBytes);
+            mma_ts(tmem + 2 * kBlockN + t * D, tmem + t * kBlockN + kk * 8, db, kIdPV, (acc || kk > 0) ? 1u : 0u);
+          }
+        };
+        if (n0 > 0 && !mbar_wait(q_full(0), 0, abort_flag)) ok = false;
+        if (n1 > 0 && !mbar_wait(q_full(1), 0, abort_flag)) ok = false;
+        if (ok && n_max > 0) {
+          if (!mbar_wait(kv_full(0), 0, abort_flag)) {
+            ok = false;
+          } else {
+            tc_fence_after();
+            if (n0 > 0) {
+              issue_s(0, 0);
+              mma_commit(s_full(0));
+            }
+            if (n1 > 0) {
+              issue_s(1, 0);
+              mma_commit(s_full(1));
+            }
+            mma_commit(kv_empty(0));
+          }
+        }
+#pragma unroll 1
+        for (int j = 0; ok && j < n_max; ++j) {
+          const int itv = 2 * j + 1;
+          const int slot_v = itv % NS;
+          const int itk = 2 * j + 2;
+          const int slot_k = itk % NS;
+          if (!mbar_wait(kv_full(slot_v), (itv / NS) & 1, abort_flag)) break;
+          bool k_ready = false;
+#pragma unroll 1
+          for (int t = 0; t < 2; ++t) {
+            const int nt = t ? n1 : n0;
+            if (j >= nt) continue;
+            if (!mbar_wait(p_full(t), j & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            const bool more = j + 1 < nt;
+            if (more && !k_ready) {
+              if (!mbar_wait(kv_full(slot_k), (itk / NS) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              k_ready = true;
+            }
+            tc_fence_after();
+            issue_pv(t, slot_v, j > 0);
+            if (more) {
+              issue_s(t, slot_k);
+              mma_commit(s_full(t));
+            } else {
+              mma_commit(o_full(t));
+            }
+          }
+          if (!ok) break;
+          mma_commit(kv_empty(slot_v));
+          if (k_ready) mma_commit(kv_empty(slot_k));
+        }
+        // Every MMA this thread issued must finish before TMEM is released.
+        mma_commit(drain);
+        mbar_wait_drain(drain, 0);
+      }
+      __syncwarp();
+    }
+  } else {
+    // Warpgroups 0 and 1: softmax / epilogue for query tile 0 and 1.
+    regs_increase<kSoftmaxRegs>();
+    const int t = warp >> 2;      // query tile 0 or 1
+    const int wq = warp & 3;      // TMEM lane quarter of this warp
+    const int r_in_tile = wq * 32 + lane;
+    const int row0 = t ? row0_1 : row0_0;
+    const int row = row0 + r_in_tile;
+    const int n = t ? n1 : n0;
+    const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_bits + t * kBlockN;
+    const uint32_t tO = tmem + lane_bits + 2 * kBlockN + t * D;
+    const float c = p.scale_log2;
+    const int row_limit = p.causal ? row + p.causal_offset : INT_MAX - kBlockN;
+    float m_used = -INFINITY;
+    float l = 0.f;
+    bool ok = true;
+
+#pragma unroll 1
+    for (int j = 0; j < n; ++j) {
+      if (!mbar_wait(s_full(t), j & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t s[4][32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, s[q]);
+      tmem_wait_ld();
+
+      const int k0 = j * kBlockN;
+      const bool need_mask = (k0 + kBlockN > p.Sk) || (p.causal && k0 + kBlockN - 1 > row0 + p.causal_offset);
+      if (need_mask) {
+        const int lim = min(p.Sk - 1, row_limit) - k0;  // last visible column
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (q * 32 + e > lim) s[q][e] = __float_as_uint(-INFINITY);
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        mx0 = fmaxf(mx0, __uint_as_float(s[0][e]));
+        mx1 = fmaxf(mx1, __uint_as_float(s[1][e]));
+        mx2 = fmaxf(mx2, __uint_as_float(s[2][e]));
+        mx3 = fmaxf(mx3, __uint_as_float(s[3][e]));
+      }
+      const float m_new = fmaxf(m_used, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)));
+      // (m_new - m_used) is NaN while both are -inf: no rescale then.
+      const bool rescale = (m_new - m_used) * c > kRescaleThreshold;
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = ex2_approx((m_used - m_new) * c);
+        m_used = m_new;
+        l *= alpha;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t o[32];
+          tmem_ld32(tO + q * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + q * 32, o);
+        }
+      }
+      const float mc = (m_used == -INFINITY) ? 0.f : m_used * c;
+      float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float a = ex2_approx(fmaf(__uint_as_float(s[q][2 * e]), c, -mc));
+          const float bb = ex2_approx(fmaf(__uint_as_float(s[q][2 * e + 1]), c, -mc));
+          sum0 += a;
+          sum1 += bb;
+          pk[e] = pack_bf16x2(a, bb);
+        }
+        tmem_st16(tS + q * 16, pk);
+      }
+      l += sum0 + sum1;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full(t));
+    }
+
+    // ---- epilogue: O / l -> bf16 -> swizzled smem (this tile's Q buffer) -> TMA store
+    if (row0 < p.Sq) {
+      if (ok && n > 0 && !mbar_wait(o_full(t), 0, abort_flag)) ok = false;
+      tc_fence_after();
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const uint32_t stage = sQ + t * Cfg::kTileBytes;
+#pragma unroll 1
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t o[32];
+        if (ok && n > 0) {
+          tmem_ld32(tO + q * 32, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+#pragma unroll
+        for (int c16 = 0; c16 < 4; ++c16) {
+          const int chunk = q * 4 + c16;  // 16-byte chunk index in the row (8 bf16 each)
+          const int blk = chunk >> 3;
+          const int cw = (chunk & 7) ^ (r_in_tile & 7);
+          const uint32_t addr = stage + blk * Cfg::kBlockBytes + r_in_tile * 128 + cw * 16;
+          const uint32_t* f = &o[c16 * 8];
+          st_shared_v4(addr,
+                       pack_bf16x2(__uint_as_float(f[0]) * inv_l, __uint_as_float(f[1]) * inv_l),
+                       pack_bf16x2(__uint_as_float(f[2]) * inv_l, __uint_as_float(f[3]) * inv_l),
+                       pack_bf16x2(__uint_as_float(f[4]) * inv_l, __uint_as_float(f[5]) * inv_l),
+                       pack_bf16x2(__uint_as_float(f[6]) * inv_l, __uint_as_float(f[7]) * inv_l));
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1 + t, 128);
+      if (r_in_tile == 0) {
+        for (int blk = 0; blk < Cfg::kBlocks; ++blk)
+          tma_store_3d(&p.tm_o, stage + blk * Cfg::kBlockBytes, blk * 64, row0, bh);
+        bulk_commit_group();
+        bulk_wait_group0();
+      }
+      if (p.lse != nullptr && row < p.Sq) {
+        const float lse = (l > 0.f) ? (m_used * p.scale + lg2_approx(l) * 0.69314718055994531f) : -INFINITY;
+        p.lse[static_cast<int64_t>(bh) * p.Sq + row] = lse;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace sdpa

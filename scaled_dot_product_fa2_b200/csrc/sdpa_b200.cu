@@ -1,0 +1,393 @@
+// sdpa_b200.cu -- host side of libsdpa_b200.so: argument checks, TMA
+// descriptors, launch configuration and the extern "C" entry points declared
+// in include/sdpa_b200.h.  Device code lives in prefill.cuh and decode.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "sdpa_b200.h"
+#include "decode.cuh"
+#include "prefill.cuh"
+
+namespace sdpa {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxSeq = 1 << 30;
+
+// ------------------------------------------------------------ checks
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+attn_status_t check_common(const void* q, const void* k, const void* v, const void* o, const float* lse, int B,
+                           int Hq, int Hkv, int Sq, int Sk, int d, float scale, int causal) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Sq < 0 || Sk < 0 || d <= 0) return ATTN_ERR_SHAPE;
+  if (Sq > kMaxSeq || Sk > kMaxSeq) return ATTN_ERR_SHAPE;
+  if (static_cast<int64_t>(B) * Hq > INT_MAX / 4) return ATTN_ERR_SHAPE;
+  if (Hq % Hkv != 0) return ATTN_ERR_GQA;
+  if (d != 64 && d != 128) return ATTN_ERR_HEADDIM;
+  if (causal < ATTN_CAUSAL_NONE || causal > ATTN_CAUSAL_BOTTOM_RIGHT) return ATTN_ERR_CAUSAL;
+  if (!(scale >= 0.f) || std::isinf(scale)) return ATTN_ERR_SCALE;  // also rejects NaN
+  const bool empty = (B == 0 || Sq == 0);
+  if (!empty) {
+    if (q == nullptr || o == nullptr) return ATTN_ERR_NULL;
+    if (Sk > 0 && (k == nullptr || v == nullptr)) return ATTN_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(o, 16)) return ATTN_ERR_ALIGN;
+    if (Sk > 0 && (!aligned(k, 16) || !aligned(v, 16))) return ATTN_ERR_ALIGN;
+    if (lse != nullptr && !aligned(lse, 4)) return ATTN_ERR_ALIGN;
+  }
+  return ATTN_OK;
+}
+
+float effective_scale(float scale, int d) { return scale == 0.f ? 1.f / std::sqrt(static_cast<float>(d)) : scale; }
+
+int causal_offset(int causal, int Sq, int Sk) { return causal == ATTN_CAUSAL_BOTTOM_RIGHT ? Sk - Sq : 0; }
+
+// ------------------------------------------------------------ device info
+struct DeviceInfo {
+  bool probed = false;
+  bool ok = false;
+  int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+attn_status_t current_device(int* dev_out, int* sms_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    di.probed = true;
+    di.ok = (major == 10 && minor == 0);
+    di.sms = sms;
+  }
+  if (!di.ok) return ATTN_ERR_ARCH;
+  if (dev_out) *dev_out = dev;
+  if (sms_out) *sms_out = di.sms;
+  return ATTN_OK;
+}
+
+// Best-effort SM count for size queries that may run without a device.
+int sm_count_or_default() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+    return sms;
+  cudaGetLastError();  // clear a sticky "no device" error from the probe
+  return 148;
+}
+
+// ------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 map over a contiguous [outer][rows][d] tensor; box = {64, box_rows, 1},
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_map(CUtensorMap* map, const void* base, int d, int rows, int64_t outer, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(outer)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(rows) * d * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------ kernels' config
+constexpr int kStagesD128 = 4;
+constexpr int kStagesD64 = 8;
+constexpr int kDecStages = 3;   // 3 x 32 KB ring: two decode CTAs fit on one SM
+constexpr int kDecCtasPerSm = 2;
+
+template <typename K>
+bool set_smem(K kernel, int bytes, int dev, bool* done) {
+  if (done[dev]) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  done[dev] = true;
+  return true;
+}
+
+// Fill o with zeros and lse with -inf (rows with no visible key, Sk == 0).
+__global__ void fill_empty_kernel(uint16_t* o, float* lse, int64_t rows, int d) {
+  const int64_t n = rows * d;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    o[i] = 0;
+    if (lse != nullptr && i % d == 0) lse[i / d] = -INFINITY;
+  }
+}
+
+attn_status_t launch_fill_empty(void* o, float* lse, int64_t rows, int d, cudaStream_t st) {
+  const int64_t n = rows * d;
+  const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096));
+  fill_empty_kernel<<<blocks, 256, 0, st>>>(static_cast<uint16_t*>(o), lse, rows, d);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, int NS>
+attn_status_t launch_prefill(const PrefillParams& prm, int grid, int dev, cudaStream_t st) {
+  static bool smem_done[kMaxDevices] = {};
+  static std::mutex mu;
+  using Cfg = PrefillCfg<D, NS>;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!smem_done[dev]) {
+      // The kernel's in-kernel register split (setmaxnreg) adds up to exactly
+      // kLaunchRegs per thread; launching with any other allocation could make
+      // setmaxnreg.inc wait forever, so refuse instead.
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, prefill_kernel<D, NS>) != cudaSuccess || fa.numRegs != kLaunchRegs)
+        return ATTN_ERR_CUDA;
+    }
+    if (!set_smem(prefill_kernel<D, NS>, Cfg::kSmemBytes, dev, smem_done)) return ATTN_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kPrefillThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = st;
+  return cudaLaunchKernelEx(&cfg, prefill_kernel<D, NS>, prm) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ decode split policy
+// Pick tiles-per-split so that (waves of CTAs) x (tiles per CTA + fixed cost)
+// is smallest, i.e. the SMs finish as evenly as possible.
+int decode_tiles_per_split(int64_t pairs, int total_tiles, int sms, int requested_splits) {
+  if (total_tiles <= 0) return 1;
+  if (requested_splits > 0) {
+    const int s = std::min(requested_splits, total_tiles);
+    return (total_tiles + s - 1) / s;
+  }
+  const int64_t slots = static_cast<int64_t>(sms) * kDecCtasPerSm;
+  const double fixed = 2.0;  // per-CTA start-up cost, in tiles
+  int best_t = total_tiles;
+  double best = 1e300;
+  for (int t = 1; t <= total_tiles; ++t) {
+    const int64_t splits = (total_tiles + t - 1) / t;
+    if (t > 1 && (total_tiles + t - 2) / (t - 1) == splits) continue;  // same split count, fewer tiles is better
+    const int64_t ctas = pairs * splits;
+    const int64_t waves = (ctas + slots - 1) / slots;
+    const double cost = static_cast<double>(waves) * (t + fixed);
+    if (cost < best - 1e-9) {
+      best = cost;
+      best_t = t;
+    }
+  }
+  return best_t;
+}
+
+bool decode_shape(int B, int Hq, int Hkv, int Sq, int Sk, int d, int num_splits, int sms, int* tiles_per_split,
+                  int* nsplit, int* row_groups) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || Sk <= 0 || (d != 64 && d != 128) || Hq % Hkv != 0) return false;
+  if (Sq > kMaxSeq || Sk > kMaxSeq || num_splits < 0) return false;
+  const int group = Hq / Hkv;
+  const int64_t rows = static_cast<int64_t>(group) * Sq;
+  const int rg = static_cast<int>((rows + kDecRows - 1) / kDecRows);
+  const int total_tiles = (Sk + kDecKeys - 1) / kDecKeys;
+  const int64_t pairs = static_cast<int64_t>(B) * Hkv * rg;
+  const int t = decode_tiles_per_split(pairs, total_tiles, sms, num_splits);
+  *tiles_per_split = t;
+  *nsplit = (total_tiles + t - 1) / t;
+  *row_groups = rg;
+  return true;
+}
+
+size_t decode_ws_bytes(int B, int Hq, int Sq, int d, int nsplit) {
+  const size_t rows = static_cast<size_t>(B) * Hq * Sq;
+  const size_t po = rows * nsplit * d * sizeof(float);
+  return po + rows * nsplit * sizeof(float2);
+}
+
+template <int D>
+attn_status_t launch_decode(const DecodeParams& prm, int grid, float* part_o, float2* part_ml, void* o, float* lse,
+                            int64_t rows, int dev, cudaStream_t st) {
+  static bool smem_done[kMaxDevices] = {};
+  static std::mutex mu;
+  using Cfg = DecodeCfg<D, kDecStages>;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!set_smem(decode_split_kernel<D, kDecStages>, Cfg::kSmemBytes, dev, smem_done)) return ATTN_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = st;
+  if (cudaLaunchKernelEx(&cfg, decode_split_kernel<D, kDecStages>, prm) != cudaSuccess) return ATTN_ERR_CUDA;
+  const int cgrid = static_cast<int>((rows + 3) / 4);
+  decode_combine_kernel<D><<<cgrid, 128, 0, st>>>(part_o, part_ml, static_cast<uint16_t*>(o), lse, rows,
+                                                   prm.nsplit);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace sdpa
+
+using namespace sdpa;
+
+extern "C" {
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                       int Sq, int Sk, int d, float scale, int causal, void* stream) {
+  attn_status_t s = check_common(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
+  if (s != ATTN_OK) return s;
+  if (B == 0 || Sq == 0) return ATTN_OK;
+  int dev = 0;
+  if ((s = current_device(&dev, nullptr)) != ATTN_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t rows = static_cast<int64_t>(B) * Hq * Sq;
+  if (Sk == 0) return launch_fill_empty(o, lse, rows, d, st);
+
+  const float sc = effective_scale(scale, d);
+  PrefillParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  if (!make_map(&prm.tm_q, q, d, Sq, static_cast<int64_t>(B) * Hq, kBlockM) ||
+      !make_map(&prm.tm_k, k, d, Sk, static_cast<int64_t>(B) * Hkv, kBlockN) ||
+      !make_map(&prm.tm_v, v, d, Sk, static_cast<int64_t>(B) * Hkv, kBlockN) ||
+      !make_map(&prm.tm_o, o, d, Sq, static_cast<int64_t>(B) * Hq, kBlockM))
+    return ATTN_ERR_CUDA;
+  prm.lse = lse;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.Sq = Sq;
+  prm.Sk = Sk;
+  prm.group = Hq / Hkv;
+  prm.causal = causal;
+  prm.causal_offset = causal_offset(causal, Sq, Sk);
+  prm.num_units = (Sq + 2 * kBlockM - 1) / (2 * kBlockM);
+  prm.lpt = causal != ATTN_CAUSAL_NONE ? 1 : 0;
+  prm.scale = sc;
+  prm.scale_log2 = sc * 1.4426950408889634f;
+  const int64_t grid = static_cast<int64_t>(B) * Hq * prm.num_units;
+  if (grid > INT_MAX) return ATTN_ERR_SHAPE;
+  if (d == 128) return launch_prefill<128, kStagesD128>(prm, static_cast<int>(grid), dev, st);
+  return launch_prefill<64, kStagesD64>(prm, static_cast<int>(grid), dev, st);
+}
+
+int attn_decode_num_splits(int B, int Hq, int Hkv, int Sq, int Sk, int d) {
+  int t = 0, ns = 0, rg = 0;
+  if (!decode_shape(B, Hq, Hkv, Sq, Sk, d, 0, sm_count_or_default(), &t, &ns, &rg)) return 0;
+  return ns;
+}
+
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int d, int num_splits) {
+  int t = 0, ns = 0, rg = 0;
+  const int sms = num_splits > 0 ? 148 : sm_count_or_default();
+  if (!decode_shape(B, Hq, Hkv, Sq, Sk, d, num_splits, sms, &t, &ns, &rg)) return 0;
+  return decode_ws_bytes(B, Hq, Sq, d, ns);
+}
+
+attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                                  int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale, int causal,
+                                  int num_splits, void* workspace, size_t workspace_bytes, void* stream) {
+  attn_status_t s = check_common(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
+  if (s != ATTN_OK) return s;
+  if (num_splits < 0) return ATTN_ERR_SHAPE;
+  if (B == 0 || Sq == 0) return ATTN_OK;
+  int dev = 0, sms = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (Sk == 0) {
+    if ((s = current_device(&dev, &sms)) != ATTN_OK) return s;
+    return launch_fill_empty(o, lse, static_cast<int64_t>(B) * Hq * Sq, d, st);
+  }
+  int t = 0, ns = 0, rg = 0;
+  // The split policy must not depend on the device when the caller fixed the count.
+  const int sms_for_policy = num_splits > 0 ? 148 : sm_count_or_default();
+  if (!decode_shape(B, Hq, Hkv, Sq, Sk, d, num_splits, sms_for_policy, &t, &ns, &rg)) return ATTN_ERR_SHAPE;
+  const size_t need = decode_ws_bytes(B, Hq, Sq, d, ns);
+  if (workspace == nullptr || !aligned(workspace, 16) || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  if ((s = current_device(&dev, &sms)) != ATTN_OK) return s;
+
+  const float sc = effective_scale(scale, d);
+  const int64_t rows = static_cast<int64_t>(B) * Hq * Sq;
+  DecodeParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  if (!make_map(&prm.tm_k, k_cache, d, Sk, static_cast<int64_t>(B) * Hkv, kDecKeys) ||
+      !make_map(&prm.tm_v, v_cache, d, Sk, static_cast<int64_t>(B) * Hkv, kDecKeys))
+    return ATTN_ERR_CUDA;
+  float* part_o = static_cast<float*>(workspace);
+  float2* part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + rows * ns * d * sizeof(float));
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.part_o = part_o;
+  prm.part_ml = part_ml;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.Sq = Sq;
+  prm.Sk = Sk;
+  prm.group = Hq / Hkv;
+  prm.causal = causal;
+  prm.causal_offset = causal_offset(causal, Sq, Sk);
+  prm.nsplit = ns;
+  prm.tiles_per_split = t;
+  prm.row_groups = rg;
+  prm.scale = sc;
+  prm.scale_log2 = sc * 1.4426950408889634f;
+  const int64_t grid = static_cast<int64_t>(B) * Hkv * ns * rg;
+  if (grid > INT_MAX || (rows + 3) / 4 > INT_MAX) return ATTN_ERR_SHAPE;
+  if (d == 128) return launch_decode<128>(prm, static_cast<int>(grid), part_o, part_ml, o, lse, rows, dev, st);
+  return launch_decode<64>(prm, static_cast<int>(grid), part_o, part_ml, o, lse, rows, dev, st);
+}
+
+const char* attn_status_string(attn_status_t status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_NULL: return "a required pointer is NULL";
+    case ATTN_ERR_SHAPE: return "invalid or unsupported size";
+    case ATTN_ERR_GQA: return "Hq is not a multiple of Hkv";
+    case ATTN_ERR_HEADDIM: return "head_dim must be 64 or 128";
+    case ATTN_ERR_ALIGN: return "pointer not aligned (16 bytes; lse 4 bytes)";
+    case ATTN_ERR_CAUSAL: return "unknown causal mode";
+    case ATTN_ERR_WORKSPACE: return "decode workspace missing, misaligned or too small";
+    case ATTN_ERR_CUDA: return "a CUDA runtime call failed";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel gave up";
+    case ATTN_ERR_ARCH: return "the current device is not sm_100 (B200)";
+    case ATTN_ERR_SCALE: return "scale must be 0 (default) or finite and > 0";
+  }
+  return "unknown status";
+}
+
+attn_status_t attn_check_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, sdpa::g_error_word, sizeof(word)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(sdpa::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+    return ATTN_ERR_DEVICE_TIMEOUT;
+  }
+  return ATTN_OK;
+}
+
+int attn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,124 @@
+"""Torch-facing wrappers over the C ABI (argument marshalling only).
+
+Every computation happens in the CUDA kernels of libsdpa_b200.so; these
+functions only check dtypes/devices, allocate outputs with torch and pass raw
+pointers plus the current CUDA stream.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+
+CAUSAL_NONE, CAUSAL_TOP_LEFT, CAUSAL_BOTTOM_RIGHT = 0, 1, 2
+
+
+def _stream_handle(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check_tensor(name: str, t: torch.Tensor, dtype: torch.dtype, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _shapes(q, k, v):
+    _check_tensor("q", q, torch.bfloat16, 4)
+    _check_tensor("k", k, torch.bfloat16, 4)
+    _check_tensor("v", v, torch.bfloat16, 4)
+    B, Hq, Sq, d = q.shape
+    Bk, Hkv, Sk, dk = k.shape
+    if Bk != B or dk != d or tuple(v.shape) != tuple(k.shape):
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    if not (q.device == k.device == v.device):
+        raise ValueError("q, k, v must be on one device")
+    return B, Hq, Hkv, Sq, Sk, d
+
+
+def _outputs(q, out, lse, want_lse):
+    B, Hq, Sq, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_tensor("out", out, torch.bfloat16, 4)
+        if tuple(out.shape) != tuple(q.shape):
+            raise ValueError("out must have the shape of q")
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _check_tensor("lse", lse, torch.float32, 3)
+        if tuple(lse.shape) != (B, Hq, Sq):
+            raise ValueError("lse must be [B, Hq, Sq]")
+    return out, lse
+
+
+def attn_fwd(q, k, v, causal: int = CAUSAL_NONE, scale: float = 0.0, out=None, lse=None,
+             return_lse: bool = True):
+    """O = softmax(scale * q k^T + mask) v through ``attn_fwd`` of the C ABI.
+
+    q [B,Hq,Sq,d], k/v [B,Hkv,Sk,d] bf16 contiguous CUDA tensors; ``scale=0``
+    means 1/sqrt(d).  Returns (o, lse) with lse fp32 [B,Hq,Sq] (None when
+    ``return_lse`` is False and no ``lse`` buffer was given).
+    """
+    B, Hq, Hkv, Sq, Sk, d = _shapes(q, k, v)
+    out, lse = _outputs(q, out, lse, return_lse)
+    lib = _lib.get()
+    with torch.cuda.device(q.device):
+        st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                          lse.data_ptr() if lse is not None else None,
+                          B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal), _stream_handle(q.device))
+    _lib.check(st, "attn_fwd")
+    return out, lse
+
+
+def decode_num_splits(B, Hq, Hkv, Sq, Sk, d) -> int:
+    return int(_lib.get().attn_decode_num_splits(B, Hq, Hkv, Sq, Sk, d))
+
+
+def decode_workspace_size(B, Hq, Hkv, Sq, Sk, d, num_splits: int = 0) -> int:
+    return int(_lib.get().attn_decode_workspace_size(B, Hq, Hkv, Sq, Sk, d, num_splits))
+
+
+def decode_workspace(q, k_cache, num_splits: int = 0) -> torch.Tensor:
+    """A caller-owned workspace buffer sized for ``attn_decode_splitkv``."""
+    B, Hq, Sq, d = q.shape
+    Hkv, Sk = k_cache.shape[1], k_cache.shape[2]
+    with torch.cuda.device(q.device):
+        n = decode_workspace_size(B, Hq, Hkv, Sq, Sk, d, num_splits)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+
+
+def attn_decode_splitkv(q, k_cache, v_cache, causal: int = CAUSAL_BOTTOM_RIGHT, scale: float = 0.0,
+                        num_splits: int = 0, workspace=None, out=None, lse=None, return_lse: bool = True):
+    """Split-KV decode through ``attn_decode_splitkv`` of the C ABI.  Returns (o, lse)."""
+    B, Hq, Hkv, Sq, Sk, d = _shapes(q, k_cache, v_cache)
+    out, lse = _outputs(q, out, lse, return_lse)
+    if workspace is None:
+        workspace = decode_workspace(q, k_cache, num_splits)
+    if workspace.device != q.device or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous buffer on q's device")
+    lib = _lib.get()
+    with torch.cuda.device(q.device):
+        st = lib.attn_decode_splitkv(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
+                                     lse.data_ptr() if lse is not None else None,
+                                     B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal), int(num_splits),
+                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                     _stream_handle(q.device))
+    _lib.check(st, "attn_decode_splitkv")
+    return out, lse
+
+
+def check_device_error(device=None) -> None:
+    """Synchronize the current stream and raise if a kernel gave up on a bounded wait."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        st = _lib.get().attn_check_device_error(_stream_handle(dev))
+    _lib.check(st, "attn_check_device_error")

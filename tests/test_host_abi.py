@@ -1,0 +1,114 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The library must load on a machine without a GPU, export every function the
+header declares, and reject bad arguments on the host before touching CUDA.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from scaled_dot_product_fa2_b200 import _lib, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "sdpa_b200.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.get()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(attn_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_documented_entry_points():
+    names = declared_functions()
+    for required in ("attn_fwd", "attn_decode_splitkv", "attn_decode_workspace_size",
+                     "attn_status_string", "attn_check_device_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert names
+    raw = ctypes.CDLL(_lib.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), f"{n} declared in sdpa_b200.h but not exported"
+    assert set(_lib.EXPORTS) <= set(names)
+
+
+def test_status_strings(lib):
+    for code in range(12):
+        assert lib.attn_status_string(code)
+    assert lib.attn_status_string(0) == b"ok"
+
+
+# Fake, well-aligned device addresses: validation must fail before any use.
+P = 1 << 20
+
+
+def fwd(lib, q=P, k=P, v=P, o=P, lse=None, B=1, Hq=2, Hkv=2, Sq=8, Sk=8, d=128, scale=0.0, causal=0):
+    return lib.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(o=None), 1), (dict(k=None), 1), (dict(v=None), 1),
+    (dict(B=-1), 2), (dict(Sq=-3), 2), (dict(Sk=-1), 2), (dict(Hq=0), 2), (dict(Hkv=0), 2),
+    (dict(Sq=(1 << 30) + 1), 2),
+    (dict(Hq=6, Hkv=4), 3),
+    (dict(d=96), 4), (dict(d=256), 4), (dict(d=32), 4),
+    (dict(q=P + 8), 5), (dict(k=P + 2), 5), (dict(o=P + 4), 5), (dict(lse=P + 2), 5),
+    (dict(causal=3), 6), (dict(causal=-1), 6),
+    (dict(scale=-0.5), 11), (dict(scale=float("nan")), 11), (dict(scale=float("inf")), 11),
+])
+def test_fwd_rejects_bad_arguments_on_host(lib, kw, status):
+    assert fwd(lib, **kw) == status
+
+
+def test_fwd_empty_problem_is_ok_without_launch(lib):
+    assert fwd(lib, B=0, q=None, k=None, v=None, o=None) == 0
+    assert fwd(lib, Sq=0, q=None, k=None, v=None, o=None) == 0
+
+
+def test_decode_workspace_size_formula(lib):
+    # fixed split count: rows * splits * (d floats + 2 floats)
+    B, Hq, Hkv, Sq, Sk, d = 8, 32, 8, 4, 8192, 128
+    for splits in (1, 2, 7, 128):
+        n = lib.attn_decode_workspace_size(B, Hq, Hkv, Sq, Sk, d, splits)
+        tiles = (Sk + 63) // 64
+        t = -(-tiles // min(splits, tiles))
+        eff = -(-tiles // t)
+        assert n == B * Hq * Sq * eff * (d + 2) * 4
+    # more splits than tiles are clamped to one tile per split
+    assert lib.attn_decode_workspace_size(1, 1, 1, 1, 100, 64, 50) == 1 * 2 * (64 + 2) * 4
+    assert lib.attn_decode_workspace_size(1, 3, 2, 1, 100, 64, 1) == 0  # Hq % Hkv != 0
+    assert lib.attn_decode_workspace_size(1, 2, 2, 1, 100, 96, 1) == 0  # bad d
+    assert lib.attn_decode_num_splits(8, 32, 8, 4, 8192, 128) >= 1
+
+
+def test_decode_rejects_bad_workspace_on_host(lib):
+    args = dict(B=2, Hq=4, Hkv=2, Sq=1, Sk=256, d=128)
+    need = lib.attn_decode_workspace_size(*args.values(), 0)
+    call = lambda ws, nbytes, splits=0: lib.attn_decode_splitkv(
+        P, P, P, P, None, *args.values(), 0.0, 2, splits, ws, nbytes, None)
+    assert call(None, need) == 7
+    assert call(P + 4, need) == 7
+    assert call(P, need - 1) == 7
+    assert lib.attn_decode_splitkv(P, P, P, P, None, 2, 4, 2, 1, 256, 128, 0.0, 2, -1, P, need, None) == 2
+    assert lib.attn_decode_splitkv(P, P, P, P, None, 2, 4, 3, 1, 256, 128, 0.0, 2, 0, P, need, None) == 3
+
+
+def test_ptxas_report_checker():
+    ok = ("ptxas info    : Compiling entry function '_ZN4sdpa14prefill_kernelILi128ELi4EEEvNS_13PrefillParamsE'\n"
+          "    0 bytes stack frame, 0 bytes spill stores, 0 bytes spill loads\n"
+          "ptxas info    : Used 168 registers, used 16 barriers\n")
+    build.check_ptxas_report(ok)
+    with pytest.raises(RuntimeError):
+        build.check_ptxas_report(ok.replace("Used 168", "Used 160"))
+    with pytest.raises(RuntimeError):
+        build.check_ptxas_report(ok.replace("0 bytes spill stores", "8 bytes spill stores"))
