@@ -48,6 +48,9 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-breakdown", action="store_true", help="time the headline step only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", metavar="WORKLOAD", default=None,
+                    help="run a few untimed calls of one named workload (for ncu captures) and exit")
+    ap.add_argument("--profile-calls", type=int, default=3)
     return ap.parse_args()
 
 
@@ -158,12 +161,19 @@ def barrier(world):
 
 
 def max_over_ranks(world, x: float) -> float:
+    """Largest x over all ranks (the slowest rank's time)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(world: int, flops_per_rank_step: float, steps: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank did the same per-GPU work in at most max_ms."""
+    return world * flops_per_rank_step * steps / (max_ms / 1e3) / 1e12
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
@@ -303,6 +313,8 @@ def main():
         # the CPU oracle arm needs no process group: rank 0 runs, the others exit
         return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
     world, rank, local = setup_dist(args)
+    if args.profile:
+        return run_profile_case(args)
     import scaled_dot_product_fa2_b200 as sdpa
     from scaled_dot_product_fa2_b200 import build
     if rank == 0:
@@ -350,7 +362,7 @@ def main():
     kernel_ms = max_over_ranks(world, kernel_ms)
     wall = max_over_ranks(world, wall)
     ms_per_step = kernel_ms / args.steps
-    value = world * flops_step * args.steps / (kernel_ms / 1e3) / 1e12
+    value = weak_scaling_value(world, flops_step, args.steps, kernel_ms)
 
     # ---- end to end through the public API with host buffers (pinned), same metric
     for _ in range(2):
@@ -367,7 +379,7 @@ def main():
     e_b.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(world, e_a.elapsed_time(e_b))
-    e2e_value = world * flops_step * args.steps / (e2e_ms / 1e3) / 1e12
+    e2e_value = weak_scaling_value(world, flops_step, args.steps, e2e_ms)
     h2d = sum(s.h2d_bytes() for s in shapes)
     d2h = sum(s.d2h_bytes() for s in shapes)
 
@@ -442,6 +454,20 @@ def measure_breakdown(flush, peak_tf, hbm_gbs, rank, reps: int = 10):
         del s
     torch.cuda.empty_cache()
     return out
+
+
+def run_profile_case(args):
+    """A few back-to-back calls of one workload with an L2 flush before each:
+    the small, self-terminating command that ncu captures are taken on."""
+    import scaled_dot_product_fa2_b200 as sdpa
+    w = inputs.BY_NAME[args.profile]
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    runner = GpuDecode(w, 0) if w.decode else GpuPrefill(w, 0)
+    for _ in range(args.profile_calls):
+        flush_buf.fill_(1)
+        runner.run()
+    sdpa.check_device_error()
+    print(f"profile case {w.name}: {args.profile_calls} calls ok", flush=True)
 
 
 def run_reference(args, world, rank):
