@@ -33,9 +33,9 @@
  * aligned device pointers; lse 4-byte aligned.
  *
  * Ownership: the caller allocates and owns every buffer, including the
- * decode workspace.  The library allocates no device memory per call (one
- * 4-byte device error word per process, and nothing else) and keeps no
- * per-call search.  Calls are asynchronous on `stream` (a cudaStream_t
+ * decode workspace.  The library allocates no device memory per call (its
+ * only device memory is a 4-byte error word and the fixed scratch array of
+ * attn_decode_splitkv_static, both static) and keeps no per-call search.  Calls are asynchronous on `stream` (a cudaStream_t
  * passed as void*; NULL = legacy default stream) and never synchronize.
  *
  * Errors: argument errors are detected on the host before anything is
@@ -67,7 +67,9 @@ typedef enum {
   ATTN_ERR_CUDA = 8,           /* a CUDA runtime call failed */
   ATTN_ERR_DEVICE_TIMEOUT = 9, /* a bounded wait inside a kernel gave up */
   ATTN_ERR_ARCH = 10,          /* the current device is not compute capability 10.0 */
-  ATTN_ERR_SCALE = 11          /* scale is negative, NaN or infinite */
+  ATTN_ERR_SCALE = 11,         /* scale is negative, NaN or infinite */
+  ATTN_ERR_SCRATCH_LIMIT = 12  /* attn_decode_splitkv_static: problem needs more than
+                                  ATTN_STATIC_SCRATCH_BYTES of scratch */
 } attn_status_t;
 
 enum { ATTN_CAUSAL_NONE = 0, ATTN_CAUSAL_TOP_LEFT = 1, ATTN_CAUSAL_BOTTOM_RIGHT = 2 };
@@ -118,6 +120,34 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int d,
 attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
                                   int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale, int causal,
                                   int num_splits, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Split-KV decode that allocates nothing and takes no workspace -- for callers
+ * that cannot obtain device memory themselves: a plug-in whose host framework
+ * owns every device allocation and hands none out, or a service that fixes its
+ * memory budget at start-up and may not allocate afterwards.  Such callers
+ * cannot provide the workspace attn_decode_splitkv needs.  The pages have no
+ * counterpart to this entry point; it exists only for such callers.
+ *
+ * Same arguments, semantics and result as attn_decode_splitkv minus the
+ * workspace: the partial outputs go to a scratch array that the library keeps
+ * in device memory for the life of the process, ATTN_STATIC_SCRATCH_BYTES
+ * (16 MiB) on every GPU that loads the library.  A problem whose workspace
+ * (attn_decode_workspace_size for the same arguments) exceeds that size is
+ * rejected with ATTN_ERR_SCRATCH_LIMIT before anything is launched.
+ *
+ * The first call on each device looks up the scratch array's device address
+ * (once per device, with that device current); make that first call before
+ * any stream capture.  The scratch is shared by every call on a device and
+ * keeps the last call's contents; nothing in it needs to start at zero (each
+ * call writes every partial it later reads).  Calls that may overlap on the
+ * GPU (different streams without ordering between them) race on the scratch:
+ * order them, e.g. issue them on one stream.
+ */
+#define ATTN_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+attn_status_t attn_decode_splitkv_static(const void* q, const void* k_cache, const void* v_cache, void* o,
+                                         float* lse, int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale,
+                                         int causal, int num_splits, void* stream);
 
 /* A static, human-readable name for a status code. */
 const char* attn_status_string(attn_status_t status);

@@ -15,9 +15,10 @@
 #include "prefill.cuh"
 
 namespace sdpa {
+constexpr int kMaxDeviceSlots = 64;
 namespace {
 
-constexpr int kMaxDevices = 64;
+constexpr int kMaxDevices = kMaxDeviceSlots;
 constexpr int kMaxSeq = 1 << 30;
 
 // ------------------------------------------------------------ checks
@@ -372,6 +373,7 @@ const char* attn_status_string(attn_status_t status) {
     case ATTN_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel gave up";
     case ATTN_ERR_ARCH: return "the current device is not sm_100 (B200)";
     case ATTN_ERR_SCALE: return "scale must be 0 (default) or finite and > 0";
+    case ATTN_ERR_SCRATCH_LIMIT: return "problem needs more than the library's static decode scratch (16 MiB)";
   }
   return "unknown status";
 }
@@ -391,3 +393,47 @@ attn_status_t attn_check_device_error(void* stream) {
 int attn_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- allocation-free decode
+// Scratch for attn_decode_splitkv_static: a file-scope device array, so the
+// library never allocates on behalf of callers that may not allocate.  Every
+// device that loads the library holds it until the process exits.
+namespace {
+static __device__ __align__(256) unsigned char g_decode_static_scratch[ATTN_STATIC_SCRATCH_BYTES];
+
+void* g_static_scratch_addr[sdpa::kMaxDeviceSlots] = {};
+std::mutex g_static_scratch_mu;
+
+// Device address of the scratch array on the current device (looked up once per
+// device, with that device current).  Host code cannot use the symbol itself:
+// on the host it names a stand-in, not device memory.
+attn_status_t static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= sdpa::kMaxDeviceSlots) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (g_static_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_static_scratch) != cudaSuccess || p == nullptr) return ATTN_ERR_CUDA;
+    g_static_scratch_addr[dev] = p;
+  }
+  *out = g_static_scratch_addr[dev];
+  return ATTN_OK;
+}
+}  // namespace
+
+extern "C" attn_status_t attn_decode_splitkv_static(const void* q, const void* k_cache, const void* v_cache,
+                                                    void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Sk,
+                                                    int d, float scale, int causal, int num_splits, void* stream) {
+  attn_status_t s = check_common(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
+  if (s != ATTN_OK) return s;
+  if (num_splits < 0) return ATTN_ERR_SHAPE;
+  if (B > 0 && Sq > 0 && Sk > 0) {
+    const size_t need = attn_decode_workspace_size(B, Hq, Hkv, Sq, Sk, d, num_splits);
+    if (need == 0) return ATTN_ERR_SHAPE;
+    if (need > ATTN_STATIC_SCRATCH_BYTES) return ATTN_ERR_SCRATCH_LIMIT;
+  }
+  void* scratch = nullptr;
+  if (B > 0 && Sq > 0 && (s = static_scratch_address(&scratch)) != ATTN_OK) return s;
+  return attn_decode_splitkv(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal, num_splits, scratch,
+                             ATTN_STATIC_SCRATCH_BYTES, stream);
+}

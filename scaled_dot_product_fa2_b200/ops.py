@@ -116,6 +116,27 @@ def attn_decode_splitkv(q, k_cache, v_cache, causal: int = CAUSAL_BOTTOM_RIGHT, 
     return out, lse
 
 
+def attn_decode_splitkv_static(q, k_cache, v_cache, causal: int = CAUSAL_BOTTOM_RIGHT, scale: float = 0.0,
+                               num_splits: int = 0, out=None, lse=None, return_lse: bool = True):
+    """Split-KV decode without a workspace (``attn_decode_splitkv_static``).
+
+    For callers that cannot hand the library device memory: the partials live
+    in the library's fixed 16 MiB scratch array.  Output tensors are still the
+    caller's (allocated here with torch when not given).  Calls that may
+    overlap on the GPU share that scratch and race; issue them on one stream.
+    """
+    B, Hq, Hkv, Sq, Sk, d = _shapes(q, k_cache, v_cache)
+    out, lse = _outputs(q, out, lse, return_lse)
+    lib = _lib.get()
+    with torch.cuda.device(q.device):
+        st = lib.attn_decode_splitkv_static(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
+                                            lse.data_ptr() if lse is not None else None,
+                                            B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal), int(num_splits),
+                                            _stream_handle(q.device))
+    _lib.check(st, "attn_decode_splitkv_static")
+    return out, lse
+
+
 def check_device_error(device=None) -> None:
     """Synchronize the current stream and raise if a kernel gave up on a bounded wait."""
     dev = torch.device("cuda") if device is None else torch.device(device)
