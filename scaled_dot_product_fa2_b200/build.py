@@ -1,8 +1,9 @@
 """Build libsdpa_b200.so in-tree with nvcc for sm_100a.
 
 Usage: ``python -m scaled_dot_product_fa2_b200.build [--force]``.  The build
-also checks ptxas' report: the prefill kernels must use exactly the register
-count their in-kernel setmaxnreg split is written for, and no kernel may spill.
+also checks ptxas' report: no kernel may spill registers, and the prefill
+kernels must launch at exactly the register count their in-kernel setmaxnreg
+split is written for.
 """
 from __future__ import annotations
 

@@ -16,18 +16,24 @@
 //       warp  8    MMA issuer (one elected thread) + TMEM owner
 //       warp  9    TMA producer (one elected thread)
 //       warps 10-11 idle
-//     The block launches at kLaunchRegs registers per thread; warpgroup 2
-//     gives registers back (kCtrlRegs) so the softmax warpgroups can hold a
-//     full 128-column S row in registers (kSoftmaxRegs).  The split adds up
-//     to exactly the launch allocation: 256*kSoftmaxRegs + 128*kCtrlRegs ==
-//     384*kLaunchRegs.
-//   * TMEM (512 columns): S0 | S1 | O0 | O1.  P (bf16) is written over the
-//     first half of its own S columns and consumed from TMEM by the P.V MMA.
-//   * K/V tiles stream through an NS-slot shared-memory ring (K_j, V_j in
-//     consecutive slots), 128-byte swizzled, filled by TMA, released by
+//     The block launches at kLaunchRegs registers per thread (3 warps per SM
+//     sub-partition); warpgroup 2 gives registers back (kCtrlRegs) and the
+//     softmax warpgroups take them (kSoftmaxRegs) to hold a full 128-column S
+//     row.  The split adds up to exactly the launch allocation:
+//     256*kSoftmaxRegs + 128*kCtrlRegs == 384*kLaunchRegs.
+//   * K/V arrive as 128-key tiles through an NS-slot shared-memory ring (K_j,
+//     V_j in consecutive slots), 128-byte swizzled, filled by TMA, released by
 //     tcgen05.commit when the MMAs reading them are done.
-//   * The two query tiles ping-pong: while softmax group 0 works on S0(j)
-//     the tensor core runs P1.V and S1(j+1), and vice versa.
+//   * TMEM (512 columns) = S0 | S1 | O0 | O1.  P (bf16) is written over the
+//     first 64 columns of its own S and read by the P.V MMA from TMEM.  The
+//     softmax hands P over in two 64-key halves, so the first half of P.V runs
+//     while the second half of the exponentials is computed; the two query
+//     tiles interleave on the tensor core (one tile's P.V and next S run while
+//     the other tile's softmax works).
+//   * Every MMA sequence is fully unrolled with compile-time descriptor
+//     offsets: a 128x128x16 tcgen05.mma then issues about every 70 cycles,
+//     the tensor core's own rate; a rolled loop around the issue costs more
+//     than the MMA itself.
 //   * Rescaling of O is skipped unless the running max grows by more than
 //     2^8 in the exp2 domain (exact: the final O/l and LSE use the same m).
 #pragma once
@@ -54,13 +60,14 @@ struct PrefillParams {
 };
 
 constexpr int kBlockM = 128;  // query rows per tile
-constexpr int kBlockN = 128;  // keys per tile
+constexpr int kBlockN = 128;  // keys per TMA tile
+constexpr int kHalfN = 64;    // keys per P hand-off (half a tile)
 constexpr int kPrefillThreads = 384;
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
-constexpr int kLaunchRegs = 168;   // 3 warps per SM sub-partition: 3*32*168 <= 16384
-constexpr int kSoftmaxRegs = 224;
-constexpr int kCtrlRegs = 56;
+constexpr int kLaunchRegs = 168;  // 3 warps per SM sub-partition: 3*32*168 <= 16384
+constexpr int kSoftmaxRegs = 216;
+constexpr int kCtrlRegs = 72;
 static_assert(256 * kSoftmaxRegs + 128 * kCtrlRegs == kPrefillThreads * kLaunchRegs,
               "register split must equal the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest P kept unrescaled
@@ -70,11 +77,12 @@ struct PrefillCfg {
   static constexpr int kTileBytes = kBlockM * D * 2;  // one Q, K or V tile (bf16)
   static constexpr int kBlocks = D / 64;               // 64-column swizzle blocks per tile
   static constexpr int kBlockBytes = kBlockM * 128;    // 16 KB per swizzle block
-  static constexpr int kNumBars = 2 + 2 * NS + 2 + 2 + 2 + 1;
+  // q_full[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2][2] o_full[2] drain
+  static constexpr int kNumBars = 2 + 2 * NS + 2 + 4 + 2 + 1;
   static constexpr int kSmemBytes = (2 + NS) * kTileBytes + kNumBars * 8 + 16 + 1024;
 };
 
-// Number of key tiles the query tile starting at row0 must visit.
+// Number of 128-key tiles the query tile starting at row0 must visit.
 __device__ __forceinline__ int kv_tiles_for(const PrefillParams& p, int row0) {
   if (row0 >= p.Sq || p.Sk <= 0) return 0;
   int last_key = p.Sk - 1;
@@ -84,6 +92,42 @@ __device__ __forceinline__ int kv_tiles_for(const PrefillParams& p, int row0) {
   }
   if (last_key < 0) return 0;
   return last_key / kBlockN + 1;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// S_t = Q_t K^T: M=128, N=128, K=D in steps of 16.  Both operands K-major with
+// 128-byte swizzle: step kk starts 32*(kk%4) bytes into a 128-byte row, and the
+// next 64-column block is 16 KB further.  `dq`, `dk` are the tiles' base
+// descriptors; the offsets are compile-time, added to the address field.
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t dq, uint64_t dk) {
+  constexpr uint32_t kId = idesc_bf16_f32(kBlockM, kBlockN, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kBlockM * 128 + (kk & 3) * 32) >> 4);
+    mma_ss(d_tmem, dq + off, dk + off, kId, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O_t (+)= P_t[:, keys kb..kb+63] V[kb..kb+63, :]: M=128, N=D, K=64 in steps of
+// 16 keys = 8 TMEM columns of packed bf16 P = 2048 bytes of V rows.  V is
+// MN-major; its two 64-column blocks are 16 KB apart (leading byte offset in
+// the base descriptor `dv`).
+template <int D, int HALF>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t dv, bool acc) {
+  constexpr uint32_t kId = idesc_bf16_f32(kBlockM, D, true);
+#pragma unroll
+  for (int k4 = 0; k4 < kHalfN / 16; ++k4) {
+    constexpr int kBase = HALF * (kHalfN / 16);
+    const int kk = kBase + k4;
+    const uint64_t off = static_cast<uint64_t>((kk * 2048) >> 4);
+    mma_ts(o_tmem, p_tmem + kk * 8, dv + off, kId, (acc || kk > 0) ? 1u : 0u);
+  }
 }
 
 template <int D, int NS>
@@ -96,13 +140,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
   const uint32_t sQ = smem_u32(smem);
   const uint32_t sKV = sQ + 2 * Cfg::kTileBytes;
   const uint32_t bar0 = sKV + NS * Cfg::kTileBytes;
-  auto q_full = [&](int t) { return bar0 + 8u * t; };                 // [2] Q_t landed
-  auto kv_full = [&](int s) { return bar0 + 8u * (2 + s); };          // [NS] slot filled
-  auto kv_empty = [&](int s) { return bar0 + 8u * (2 + NS + s); };    // [NS] slot released
-  auto s_full = [&](int t) { return bar0 + 8u * (2 + 2 * NS + t); };  // [2] S_t(j) ready (P_t.V(j-1) done)
-  auto p_full = [&](int t) { return bar0 + 8u * (4 + 2 * NS + t); };  // [2] P_t(j) written (O_t rescaled)
-  auto o_full = [&](int t) { return bar0 + 8u * (6 + 2 * NS + t); };  // [2] last P_t.V done
-  const uint32_t drain = bar0 + 8u * (8 + 2 * NS);                    // every MMA done
+  auto q_full = [&](int t) { return bar0 + 8u * t; };                               // Q_t landed
+  auto kv_full = [&](int s) { return bar0 + 8u * (2 + s); };                        // slot filled
+  auto kv_empty = [&](int s) { return bar0 + 8u * (2 + NS + s); };                  // slot released
+  auto s_full = [&](int t) { return bar0 + 8u * (2 + 2 * NS + t); };                // S_t(j) ready
+  auto p_full = [&](int t, int h) { return bar0 + 8u * (4 + 2 * NS + 2 * t + h); };  // P half written
+  auto o_full = [&](int t) { return bar0 + 8u * (8 + 2 * NS + t); };                // last P.V done
+  const uint32_t drain = bar0 + 8u * (10 + 2 * NS);                                 // every MMA done
   uint8_t* bar_ptr = smem + 2 * Cfg::kTileBytes + NS * Cfg::kTileBytes;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * Cfg::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -133,7 +177,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
     for (int t = 0; t < 2; ++t) {
       mbar_init(q_full(t), 1);
       mbar_init(s_full(t), 1);
-      mbar_init(p_full(t), 4);  // one arrive per softmax warp
+      mbar_init(p_full(t, 0), 4);  // one arrive per softmax warp
+      mbar_init(p_full(t, 1), 4);
       mbar_init(o_full(t), 1);
     }
     for (int s = 0; s < NS; ++s) {
@@ -152,7 +197,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
   if (warp >= 8) {
     // Warpgroup 2 (control): every warp runs the same setmaxnreg first.
     regs_decrease<kCtrlRegs>();
@@ -195,35 +239,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
     } else if (warp == kMmaWarp) {
       // --------------------------------------------------------- MMA issuer
       if (lane == 0) {
-        constexpr uint32_t kIdS = idesc_bf16_f32(kBlockM, kBlockN, false);
-        constexpr uint32_t kIdPV = idesc_bf16_f32(kBlockM, D, true);
-        constexpr uint32_t kHiK = sdesc_hi(1024);  // K-major: 8-row groups 1024 B apart
-        constexpr uint32_t kHiV = sdesc_hi(1024);  // MN-major: 8-key groups 1024 B apart
         bool ok = true;
-        // S_t = Q_t K^T over D in steps of 16 (32 bytes inside a 128-byte swizzle row,
-        // next 64-column block 16 KB further).
-        auto issue_s = [&](int t, int slot) {
-          const uint32_t qa = sQ + t * Cfg::kTileBytes;
-          const uint32_t ka = sKV + slot * Cfg::kTileBytes;
-#pragma unroll 1
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * Cfg::kBlockBytes + (kk & 3) * 32;
-            const uint64_t da = (static_cast<uint64_t>(kHiK) << 32) | sdesc_lo(qa + off, 16);
-            const uint64_t db = (static_cast<uint64_t>(kHiK) << 32) | sdesc_lo(ka + off, 16);
-            mma_ss(tmem + t * kBlockN, da, db, kIdS, kk > 0 ? 1u : 0u);
-          }
-        };
-        // O_t (+)= P_t V over the 128 keys in steps of 16 (8 TMEM columns of
-        // packed bf16 P; 16 rows of V = 2048 bytes).  V is MN-major: its two
-        // 64-column blocks are 16 KB apart (leading byte offset).
-        auto issue_pv = [&](int t, int slot, bool acc) {
-          const uint32_t va = sKV + slot * Cfg::kTileBytes;
-#pragma unroll 1
-          for (int kk = 0; kk < kBlockN / 16; ++kk) {
-            const uint64_t db = (static_cast<uint64_t>(kHiV) << 32) | sdesc_lo(va + kk * 2048, Cfg::kBlockBytes);
-            mma_ts(tmem + 2 * kBlockN + t * D, tmem + t * kBlockN + kk * 8, db, kIdPV, (acc || kk > 0) ? 1u : 0u);
-          }
-        };
+        const uint64_t hi = static_cast<uint64_t>(sdesc_hi(1024)) << 32;  // 8-row groups 1024 B apart
+        const uint64_t dq0 = hi | sdesc_lo(sQ, 16);
+        const uint64_t dq1 = hi | sdesc_lo(sQ + Cfg::kTileBytes, 16);
+        auto dk = [&](int slot) { return hi | sdesc_lo(sKV + slot * Cfg::kTileBytes, 16); };
+        auto dv = [&](int slot) { return hi | sdesc_lo(sKV + slot * Cfg::kTileBytes, Cfg::kBlockBytes); };
+        const uint32_t tS0 = tmem, tS1 = tmem + kBlockN;
+        const uint32_t tO0 = tmem + 2 * kBlockN, tO1 = tmem + 2 * kBlockN + D;
         if (n0 > 0 && !mbar_wait(q_full(0), 0, abort_flag)) ok = false;
         if (n1 > 0 && !mbar_wait(q_full(1), 0, abort_flag)) ok = false;
         if (ok && n_max > 0) {
@@ -231,12 +254,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
             ok = false;
           } else {
             tc_fence_after();
+            const uint64_t k0 = dk(0);
             if (n0 > 0) {
-              issue_s(0, 0);
+              issue_qk<D>(tS0, dq0, k0);
               mma_commit(s_full(0));
             }
             if (n1 > 0) {
-              issue_s(1, 0);
+              issue_qk<D>(tS1, dq1, k0);
               mma_commit(s_full(1));
             }
             mma_commit(kv_empty(0));
@@ -249,27 +273,39 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
           const int itk = 2 * j + 2;
           const int slot_k = itk % NS;
           if (!mbar_wait(kv_full(slot_v), (itv / NS) & 1, abort_flag)) break;
+          const uint64_t v_desc = dv(slot_v);
+          const uint64_t k_desc = dk(slot_k);
           bool k_ready = false;
 #pragma unroll 1
           for (int t = 0; t < 2; ++t) {
             const int nt = t ? n1 : n0;
             if (j >= nt) continue;
-            if (!mbar_wait(p_full(t), j & 1, abort_flag)) {
+            const uint32_t tO = t ? tO1 : tO0;
+            const uint32_t tS = t ? tS1 : tS0;
+            // first half of P.V as soon as the softmax has written it
+            if (!mbar_wait(p_full(t, 0), j & 1, abort_flag)) {
               ok = false;
               break;
             }
+            tc_fence_after();
+            issue_pv<D, 0>(tO, tS, v_desc, j > 0);
+            if (!mbar_wait(p_full(t, 1), j & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv<D, 1>(tO, tS, v_desc, true);
             const bool more = j + 1 < nt;
             if (more && !k_ready) {
               if (!mbar_wait(kv_full(slot_k), (itk / NS) & 1, abort_flag)) {
                 ok = false;
                 break;
               }
+              tc_fence_after();
               k_ready = true;
             }
-            tc_fence_after();
-            issue_pv(t, slot_v, j > 0);
             if (more) {
-              issue_s(t, slot_k);
+              issue_qk<D>(tS, t ? dq1 : dq0, k_desc);
               mma_commit(s_full(t));
             } else {
               mma_commit(o_full(t));
@@ -310,9 +346,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
         break;
       }
       tc_fence_after();
-      uint32_t s[4][32];
+      uint32_t sv[128];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, s[q]);
+      for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[q * 32]));
       tmem_wait_ld();
 
       const int k0 = j * kBlockN;
@@ -320,20 +356,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
       if (need_mask) {
         const int lim = min(p.Sk - 1, row_limit) - k0;  // last visible column
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (q * 32 + e > lim) s[q][e] = __float_as_uint(-INFINITY);
+        for (int e = 0; e < 128; ++e)
+          if (e > lim) sv[e] = __float_as_uint(-INFINITY);
       }
+      // row max over the 128 scores: four independent chains of 3-input max
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        mx0 = fmaxf(mx0, __uint_as_float(s[0][e]));
-        mx1 = fmaxf(mx1, __uint_as_float(s[1][e]));
-        mx2 = fmaxf(mx2, __uint_as_float(s[2][e]));
-        mx3 = fmaxf(mx3, __uint_as_float(s[3][e]));
+      for (int e = 0; e < 128; e += 8) {
+        mx0 = max3f(mx0, __uint_as_float(sv[e + 0]), __uint_as_float(sv[e + 1]));
+        mx1 = max3f(mx1, __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]));
+        mx2 = max3f(mx2, __uint_as_float(sv[e + 4]), __uint_as_float(sv[e + 5]));
+        mx3 = max3f(mx3, __uint_as_float(sv[e + 6]), __uint_as_float(sv[e + 7]));
       }
-      const float m_new = fmaxf(m_used, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)));
+      const float m_new = max3f(m_used, max3f(mx0, mx1, mx2), mx3);
       // (m_new - m_used) is NaN while both are -inf: no rescale then.
       const bool rescale = (m_new - m_used) * c > kRescaleThreshold;
       float alpha = 1.f;
@@ -342,37 +377,50 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
         m_used = m_new;
         l *= alpha;
       }
+      // O holds P.V of earlier tiles; the S wait above implies they are done.
       if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+        const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll 1
         for (int q = 0; q < D / 32; ++q) {
           uint32_t o[32];
           tmem_ld32(tO + q * 32, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          for (int e = 0; e < 32; e += 2) {
+            const float2 r = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2);
+            o[e] = __float_as_uint(r.x);
+            o[e + 1] = __float_as_uint(r.y);
+          }
           tmem_st32(tO + q * 32, o);
         }
       }
       const float mc = (m_used == -INFINITY) ? 0.f : m_used * c;
-      float sum0 = 0.f, sum1 = 0.f;
+      const float2 c2 = make_float2(c, c);
+      const float2 nmc2 = make_float2(-mc, -mc);
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t pk[16];
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float a = ex2_approx(fmaf(__uint_as_float(s[q][2 * e]), c, -mc));
-          const float bb = ex2_approx(fmaf(__uint_as_float(s[q][2 * e + 1]), c, -mc));
-          sum0 += a;
-          sum1 += bb;
-          pk[e] = pack_bf16x2(a, bb);
+        for (int e = 0; e < 64; e += 4) {
+          const int i = half * 64 + e;
+          const float2 x0 = __ffma2_rn(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), c2, nmc2);
+          const float2 x1 =
+              __ffma2_rn(make_float2(__uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3])), c2, nmc2);
+          const float2 p0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+          const float2 p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+          acc0 = __fadd2_rn(acc0, p0);
+          acc1 = __fadd2_rn(acc1, p1);
+          pk[e / 2] = pack_bf16x2(p0.x, p0.y);
+          pk[e / 2 + 1] = pack_bf16x2(p1.x, p1.y);
         }
-        tmem_st16(tS + q * 16, pk);
+        tmem_st32(tS + half * 32, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full(t, half));
       }
-      l += sum0 + sum1;
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full(t));
+      l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
     }
 
     // ---- epilogue: O / l -> bf16 -> swizzled smem (this tile's Q buffer) -> TMA store

@@ -259,7 +259,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Warpgroup-wide register reallocation (all 4 warps of a warpgroup execute it).
+// Warpgroup-wide register reallocation: every warp of a warpgroup executes the
+// same instruction, and the per-warpgroup counts must add up to the block's
+// launch allocation (otherwise setmaxnreg.inc waits for registers forever).
 template <int N>
 __device__ __forceinline__ void regs_increase() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
