@@ -64,13 +64,17 @@ def build(force: bool = False, verbose: bool = False) -> str:
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, *SOURCES]
-    proc = subprocess.run(cmd, capture_output=True, text=True)
-    if proc.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + proc.stdout + proc.stderr)
-    check_ptxas_report(proc.stdout + proc.stderr)
-    if verbose:
-        print(proc.stdout + proc.stderr)
-    os.replace(tmp, LIB)
+    try:
+        proc = subprocess.run(cmd, capture_output=True, text=True)
+        if proc.returncode != 0:
+            raise RuntimeError("nvcc failed:\n" + proc.stdout + proc.stderr)
+        check_ptxas_report(proc.stdout + proc.stderr)
+        if verbose:
+            print(proc.stdout + proc.stderr)
+        os.replace(tmp, LIB)
+    finally:
+        if os.path.exists(tmp):
+            os.remove(tmp)
     return LIB
 
 
