@@ -109,6 +109,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
   // first flattened (b*Hq + hq)*Sq + i row of this KV head
   const int64_t row_base = (static_cast<int64_t>(b) * p.Hq + static_cast<int64_t>(hkv) * p.group) * p.Sq;
 
+  // Let the combine kernel (a programmatic dependent launch) be scheduled
+  // as soon as every CTA of this grid has started; it waits for this grid's
+  // completion before it reads anything.
+  grid_dependency_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(full(s), 1);
@@ -336,6 +340,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
 // w_s = l_s exp(m_s - M), M = max_s m_s; LSE = M + ln(sum_s w_s).  A split
 // with l_s = 0 saw no visible key and gets weight 0; a row whose splits are
 // all empty gets O = 0 and LSE = -inf.
+//
+// Lane s of the warp holds split s's weight (32 splits at a time); the
+// partial rows are then read kUnroll splits at a time with independent
+// 16-byte loads, so a row costs a few memory latencies, not one per split.
+// The kernel is launched as a programmatic dependent of the split kernel: it
+// may start while the split kernel's last CTAs run, and waits for that
+// grid's completion (and the visibility of its writes) before reading.
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ part_o,
                                                              const float2* __restrict__ part_ml,
@@ -343,7 +354,9 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
                                                              int64_t rows, int nsplit) {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   constexpr int kPer = D / 32;  // floats per lane: 4 (one 16-byte load) or 2
+  constexpr int kUnroll = 8;
   constexpr float kLog2e = 1.4426950408889634f;
+  grid_dependency_wait();
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -361,22 +374,45 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
   float W = 0.f;
   if (M != -INFINITY) {
     const float* po = part_o + row * nsplit * D + lane * kPer;
-    for (int s = 0; s < nsplit; ++s) {
-      const float2 v = ml[s];
-      const float w = (v.y > 0.f) ? v.y * ex2_approx((v.x - M) * kLog2e) : 0.f;
-      W += w;
-      if constexpr (kPer == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(po + static_cast<int64_t>(s) * D);
-        acc[0] += w * x.x;
-        acc[1] += w * x.y;
-        acc[2] += w * x.z;
-        acc[3] += w * x.w;
-      } else {
-        const float2 x = *reinterpret_cast<const float2*>(po + static_cast<int64_t>(s) * D);
-        acc[0] += w * x.x;
-        acc[1] += w * x.y;
+    for (int s0 = 0; s0 < nsplit; s0 += 32) {
+      const int n = min(32, nsplit - s0);
+      float w_lane = 0.f;
+      if (lane < n) {
+        const float2 v = ml[s0 + lane];
+        w_lane = (v.y > 0.f) ? v.y * ex2_approx((v.x - M) * kLog2e) : 0.f;
+      }
+      W += w_lane;
+      for (int i0 = 0; i0 < n; i0 += kUnroll) {
+        float x[kUnroll][kPer];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          if (i0 + u < n) {
+            const float* src = po + static_cast<int64_t>(s0 + i0 + u) * D;
+            if constexpr (kPer == 4) {
+              const float4 t = *reinterpret_cast<const float4*>(src);
+              x[u][0] = t.x;
+              x[u][1] = t.y;
+              x[u][2] = t.z;
+              x[u][3] = t.w;
+            } else {
+              const float2 t = *reinterpret_cast<const float2*>(src);
+              x[u][0] = t.x;
+              x[u][1] = t.y;
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const float w = __shfl_sync(0xffffffffu, w_lane, (i0 + u) & 31);
+          if (i0 + u < n) {
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w, x[u][e], acc[e]);
+          }
+        }
       }
     }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
   }
   const float inv = (W > 0.f) ? 1.f / W : 0.f;
   uint16_t* dst = out + row * D + lane * kPer;

@@ -427,7 +427,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
     if (row0 < p.Sq) {
       if (ok && n > 0 && !mbar_wait(o_full(t), 0, abort_flag)) ok = false;
       tc_fence_after();
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      // A row whose running max is still -inf saw no visible key: O = 0 and
+      // LSE = -inf.
+      const bool empty_row = (m_used == -INFINITY) || !(l > 0.f);
+      const float inv_l = empty_row ? 0.f : 1.f / l;
       const uint32_t stage = sQ + t * Cfg::kTileBytes;
 #pragma unroll 1
       for (int q = 0; q < D / 32; ++q) {
@@ -462,7 +465,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
         bulk_wait_group0();
       }
       if (p.lse != nullptr && row < p.Sq) {
-        const float lse = (l > 0.f) ? (m_used * p.scale + lg2_approx(l) * 0.69314718055994531f) : -INFINITY;
+        const float lse = empty_row ? -INFINITY : (m_used * p.scale + lg2_approx(l) * 0.69314718055994531f);
         p.lse[static_cast<int64_t>(bh) * p.Sq + row] = lse;
       }
     }

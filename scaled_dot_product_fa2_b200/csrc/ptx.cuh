@@ -271,6 +271,16 @@ __device__ __forceinline__ void regs_decrease() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// Programmatic dependent launch: the trigger lets the next kernel on the
+// stream (launched with programmatic stream serialization) be scheduled once
+// every CTA of this grid has triggered or exited; the wait blocks until the
+// preceding grid has completed and its memory writes are visible.  Both are
+// no-ops for kernels launched without that attribute.
+__device__ __forceinline__ void grid_dependency_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

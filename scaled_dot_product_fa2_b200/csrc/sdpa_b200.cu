@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -123,7 +124,7 @@ bool make_map(CUtensorMap* map, const void* base, int d, int rows, int64_t outer
 }
 
 // ------------------------------------------------------------ kernels' config
-constexpr int kStagesD128 = 4;
+constexpr int kStagesD128 = 5;
 constexpr int kStagesD64 = 8;
 constexpr int kDecStages = 3;   // 3 x 32 KB ring: two decode CTAs fit on one SM
 constexpr int kDecCtasPerSm = 2;
@@ -179,8 +180,24 @@ attn_status_t launch_prefill(const PrefillParams& prm, int grid, int dev, cudaSt
 }
 
 // ------------------------------------------------------------ decode split policy
-// Pick tiles-per-split so that (waves of CTAs) x (tiles per CTA + fixed cost)
-// is smallest, i.e. the SMs finish as evenly as possible.
+// Pick tiles-per-split by a model of an HBM-bound grid of equal CTAs (fitted
+// to B200 measurements of the decode workload over 4..32 splits): a wave of n
+// resident CTAs with t tiles each takes t * max(n, kSatCtas) tile-times --
+// the CTAs share the HBM bandwidth, but fewer than kSatCtas CTAs cannot keep
+// it busy -- plus a fixed start-up/drain cost per wave.  In practice this
+// prefers one full wave (every CTA resident) over a short trailing wave.
+constexpr double kSatCtas = 75.0;     // CTAs that saturate HBM (per-CTA rate ~ 1/75 of the device's)
+constexpr double kWaveFixed = 330.0;  // per-wave start-up and drain, in tile-times of the whole device
+
+double decode_grid_cost(int64_t ctas, int t, int64_t slots) {
+  double cost = 0.0;
+  for (int64_t left = ctas; left > 0; left -= slots) {
+    const double n = static_cast<double>(std::min(left, slots));
+    cost += t * std::max(n, kSatCtas) + kWaveFixed;
+  }
+  return cost;
+}
+
 int decode_tiles_per_split(int64_t pairs, int total_tiles, int sms, int requested_splits) {
   if (total_tiles <= 0) return 1;
   if (requested_splits > 0) {
@@ -188,16 +205,13 @@ int decode_tiles_per_split(int64_t pairs, int total_tiles, int sms, int requeste
     return (total_tiles + s - 1) / s;
   }
   const int64_t slots = static_cast<int64_t>(sms) * kDecCtasPerSm;
-  const double fixed = 2.0;  // per-CTA start-up cost, in tiles
   int best_t = total_tiles;
   double best = 1e300;
-  for (int t = 1; t <= total_tiles; ++t) {
+  for (int t = total_tiles; t >= 1; --t) {
     const int64_t splits = (total_tiles + t - 1) / t;
-    if (t > 1 && (total_tiles + t - 2) / (t - 1) == splits) continue;  // same split count, fewer tiles is better
-    const int64_t ctas = pairs * splits;
-    const int64_t waves = (ctas + slots - 1) / slots;
-    const double cost = static_cast<double>(waves) * (t + fixed);
-    if (cost < best - 1e-9) {
+    if (t > 1 && (total_tiles + t - 2) / (t - 1) == splits) continue;  // same split count, fewer tiles each
+    const double cost = decode_grid_cost(pairs * splits, t, slots);
+    if (cost <= best * (1.0 + 1e-9)) {  // ties go to more splits (more CTAs in flight)
       best = cost;
       best_t = t;
     }
@@ -243,10 +257,24 @@ attn_status_t launch_decode(const DecodeParams& prm, int grid, float* part_o, fl
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = st;
   if (cudaLaunchKernelEx(&cfg, decode_split_kernel<D, kDecStages>, prm) != cudaSuccess) return ATTN_ERR_CUDA;
-  const int cgrid = static_cast<int>((rows + 3) / 4);
-  decode_combine_kernel<D><<<cgrid, 128, 0, st>>>(part_o, part_ml, static_cast<uint16_t*>(o), lse, rows,
-                                                   prm.nsplit);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  // The combine is a programmatic dependent launch: it may be scheduled while
+  // the split kernel's last CTAs run and waits (griddepcontrol.wait) for the
+  // split grid to complete before reading the partials.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t ccfg = {};
+  ccfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
+  ccfg.blockDim = dim3(128);
+  ccfg.dynamicSmemBytes = 0;
+  ccfg.stream = st;
+  ccfg.attrs = attr;
+  ccfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&ccfg, decode_combine_kernel<D>, static_cast<const float*>(part_o),
+                            static_cast<const float2*>(part_ml), static_cast<uint16_t*>(o), lse, rows,
+                            prm.nsplit) == cudaSuccess
+             ? ATTN_OK
+             : ATTN_ERR_CUDA;
 }
 
 }  // namespace

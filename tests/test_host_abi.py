@@ -112,3 +112,23 @@ def test_ptxas_report_checker():
         build.check_ptxas_report(ok.replace("Used 168", "Used 160"))
     with pytest.raises(RuntimeError):
         build.check_ptxas_report(ok.replace("0 bytes spill stores", "8 bytes spill stores"))
+
+
+def test_decode_split_policy_fills_one_wave(lib):
+    """The automatic split count keeps every decode CTA resident in one wave
+    when the (batch, kv head, row group) pairs alone fit in one (148 SMs x 2
+    CTAs without a device), and never makes more splits than 64-key tiles."""
+    slots = 148 * 2
+    for (B, Hq, Hkv, Sq, Sk) in [(8, 32, 8, 1, 8192), (8, 32, 8, 4, 8192), (1, 32, 8, 1, 8192),
+                                 (2, 16, 16, 1, 4096), (4, 8, 2, 2, 30000)]:
+        rg = -(-(Hq // Hkv) * Sq // 16)
+        pairs = B * Hkv * rg
+        ns = lib.attn_decode_num_splits(B, Hq, Hkv, Sq, Sk, 128)
+        tiles = -(-Sk // 64)
+        assert 1 <= ns <= tiles
+        assert pairs * ns <= slots, (B, Hq, Hkv, Sq, Sk, ns)
+    # the decode workload: 64 (batch, kv head) pairs -> 4 splits of 32 tiles, 256 CTAs
+    assert lib.attn_decode_num_splits(8, 32, 8, 1, 8192, 128) == 4
+    # more pairs than resident slots: no splitting
+    assert lib.attn_decode_num_splits(64, 32, 8, 1, 8192, 128) == 1
+
