@@ -9,13 +9,25 @@
 // block) (same notes, improvement 2: sequence-length parallelism).
 //
 // B200 mapping (this file's own design, not the pages'):
-//   * one CTA = two 128-row query tiles of one (batch, head) sharing every
-//     K/V tile it loads; 12 warps (3 warpgroups):
+//   * Persistent grid: one CTA per SM walks a static list of work units
+//     (batch*head, pair of 128-row query tiles).  For causal masks the list
+//     holds the heaviest units (the last query tiles of each head) first and
+//     is dealt to the CTAs in snake order, round by round, which balances the
+//     per-SM work like longest-processing-time-first scheduling.  One unit's
+//     epilogue overlaps the next unit's loads and first MMAs.
+//   * One CTA = two query tiles sharing every K/V tile it loads; 12 warps:
 //       warps 0-3  softmax group 0 (one thread per row of query tile 0)
 //       warps 4-7  softmax group 1 (query tile 1)
-//       warp  8    MMA issuer (one elected thread) + TMEM owner
+//       warp  8    MMA issuer for query tile 0 (one elected thread) + TMEM owner
 //       warp  9    TMA producer (one elected thread)
-//       warps 10-11 idle
+//       warp 10    MMA issuer for query tile 1
+//       warp 11    idle
+//     Each query tile has its own MMA-issuing thread.  On B200 any
+//     shared-memory access (an mbarrier wait included) by a thread that has
+//     just issued tcgen05.mma stalls it for 120-210 cycles, while only about
+//     one MMA of work is queued ahead: one issuer that waits between MMA
+//     groups starves the tensor core.  With two issuers taking turns, each
+//     one's waits overlap the other's MMAs.
 //     The block launches at kLaunchRegs registers per thread (3 warps per SM
 //     sub-partition); warpgroup 2 gives registers back (kCtrlRegs) and the
 //     softmax warpgroups take them (kSoftmaxRegs) to hold a full 128-column S
@@ -23,19 +35,21 @@
 //     256*kSoftmaxRegs + 128*kCtrlRegs == 384*kLaunchRegs.
 //   * K/V arrive as 128-key tiles through an NS-slot shared-memory ring (K_j,
 //     V_j in consecutive slots), 128-byte swizzled, filled by TMA, released by
-//     tcgen05.commit when the MMAs reading them are done.
+//     tcgen05.commit when the MMAs reading them are done.  The ring's slot
+//     sequence runs on across units.
 //   * TMEM (512 columns) = S0 | S1 | O0 | O1.  P (bf16) is written over the
 //     first 64 columns of its own S and read by the P.V MMA from TMEM.  The
-//     softmax hands P over in two 64-key halves, so the first half of P.V runs
-//     while the second half of the exponentials is computed; the two query
-//     tiles interleave on the tensor core (one tile's P.V and next S run while
-//     the other tile's softmax works).
+//     two query tiles alternate on the tensor core: one tile's P.V and next S
+//     run while the other tile's softmax works.
 //   * Every MMA sequence is fully unrolled with compile-time descriptor
 //     offsets: a 128x128x16 tcgen05.mma then issues about every 70 cycles,
 //     the tensor core's own rate; a rolled loop around the issue costs more
 //     than the MMA itself.
 //   * Rescaling of O is skipped unless the running max grows by more than
 //     2^8 in the exp2 domain (exact: the final O/l and LSE use the same m).
+//   * The epilogue writes O/l from registers straight to global memory, so a
+//     tile's Q buffer is free as soon as its last S MMA is done and the next
+//     unit's Q can load while this unit finishes.
 #pragma once
 #include <climits>
 
@@ -47,24 +61,26 @@ struct PrefillParams {
   CUtensorMap tm_q;  // [B*Hq][Sq][d] bf16, box {64, 128, 1}, 128-byte swizzle
   CUtensorMap tm_k;  // [B*Hkv][Sk][d]
   CUtensorMap tm_v;  // [B*Hkv][Sk][d]
-  CUtensorMap tm_o;  // [B*Hq][Sq][d]
+  uint16_t* o;       // [B*Hq][Sq][d] bf16 bits
   float* lse;        // [B*Hq*Sq] or nullptr
   int B, Hq, Hkv, Sq, Sk;
   int group;          // Hq / Hkv
   int causal;         // 0 none, 1 top-left, 2 bottom-right
   int causal_offset;  // key j visible to row i iff j <= i + causal_offset
-  int num_units;      // ceil(Sq / 256): CTAs per (batch, head)
-  int lpt;            // 1: launch the heaviest units first (causal)
+  int num_units;      // ceil(Sq / 256): work units per (batch, head)
+  int total_units;    // B * Hq * num_units
+  int lpt;            // 1: heaviest units first (causal)
   float scale;        // softmax scale on q.k
   float scale_log2;   // scale * log2(e)
 };
 
 constexpr int kBlockM = 128;  // query rows per tile
 constexpr int kBlockN = 128;  // keys per TMA tile
-constexpr int kHalfN = 64;    // keys per P hand-off (half a tile)
+constexpr int kHalfN = 64;    // keys per issue_pv call (half a tile)
 constexpr int kPrefillThreads = 384;
-constexpr int kMmaWarp = 8;
+constexpr int kMmaWarp = 8;    // query tile 0; also allocates and frees TMEM
 constexpr int kLoadWarp = 9;
+constexpr int kMmaWarp1 = 10;  // query tile 1
 constexpr int kLaunchRegs = 168;  // 3 warps per SM sub-partition: 3*32*168 <= 16384
 constexpr int kSoftmaxRegs = 216;
 constexpr int kCtrlRegs = 72;
@@ -77,8 +93,8 @@ struct PrefillCfg {
   static constexpr int kTileBytes = kBlockM * D * 2;  // one Q, K or V tile (bf16)
   static constexpr int kBlocks = D / 64;               // 64-column swizzle blocks per tile
   static constexpr int kBlockBytes = kBlockM * 128;    // 16 KB per swizzle block
-  // q_full[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2][2] o_full[2] drain
-  static constexpr int kNumBars = 2 + 2 * NS + 2 + 4 + 2 + 1;
+  // q_full[2] q_empty[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2] o_full[2] turn[2] drain
+  static constexpr int kNumBars = 4 + 2 * NS + 2 + 2 + 2 + 2 + 1;
   static constexpr int kSmemBytes = (2 + NS) * kTileBytes + kNumBars * 8 + 16 + 1024;
 };
 
@@ -92,6 +108,40 @@ __device__ __forceinline__ int kv_tiles_for(const PrefillParams& p, int row0) {
   }
   if (last_key < 0) return 0;
   return last_key / kBlockN + 1;
+}
+
+// The r-th work unit of CTA c in a grid of G CTAs: round r deals list entries
+// [r*G, r*G + G) in snake order (forward in even rounds, backward in odd).
+__device__ __forceinline__ int unit_index(int r, int c, int G) { return r * G + ((r & 1) ? (G - 1 - c) : c); }
+
+// Work-list entry -> (batch*head, pair index v of query tiles 2v, 2v+1).
+__device__ __forceinline__ void unit_coords(const PrefillParams& p, int idx, int& bh, int& v) {
+  const int BH = p.B * p.Hq;
+  if (p.lpt) {
+    v = p.num_units - 1 - idx / BH;
+    bh = idx % BH;
+  } else {
+    v = idx % p.num_units;
+    bh = idx / p.num_units;
+  }
+}
+
+struct Unit {
+  int bh, bhkv, row0_0, n0, n1, n_max;
+};
+
+__device__ __forceinline__ Unit make_unit(const PrefillParams& p, int idx) {
+  Unit u;
+  int v;
+  unit_coords(p, idx, u.bh, v);
+  const int b = u.bh / p.Hq;
+  const int hq = u.bh - b * p.Hq;
+  u.bhkv = b * p.Hkv + hq / p.group;
+  u.row0_0 = v * 2 * kBlockM;
+  u.n0 = kv_tiles_for(p, u.row0_0);
+  u.n1 = kv_tiles_for(p, u.row0_0 + kBlockM);
+  u.n_max = max(u.n0, u.n1);
+  return u;
 }
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -140,52 +190,38 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
   const uint32_t sQ = smem_u32(smem);
   const uint32_t sKV = sQ + 2 * Cfg::kTileBytes;
   const uint32_t bar0 = sKV + NS * Cfg::kTileBytes;
-  auto q_full = [&](int t) { return bar0 + 8u * t; };                               // Q_t landed
-  auto kv_full = [&](int s) { return bar0 + 8u * (2 + s); };                        // slot filled
-  auto kv_empty = [&](int s) { return bar0 + 8u * (2 + NS + s); };                  // slot released
-  auto s_full = [&](int t) { return bar0 + 8u * (2 + 2 * NS + t); };                // S_t(j) ready
-  auto p_full = [&](int t, int h) { return bar0 + 8u * (4 + 2 * NS + 2 * t + h); };  // P half written
-  auto o_full = [&](int t) { return bar0 + 8u * (8 + 2 * NS + t); };                // last P.V done
-  const uint32_t drain = bar0 + 8u * (10 + 2 * NS);                                 // every MMA done
+  auto q_full = [&](int t) { return bar0 + 8u * t; };                   // Q_t landed
+  auto q_empty = [&](int t) { return bar0 + 8u * (2 + t); };            // Q_t's last S MMA done
+  auto kv_full = [&](int s) { return bar0 + 8u * (4 + s); };            // slot filled
+  auto kv_empty = [&](int s) { return bar0 + 8u * (4 + NS + s); };      // slot released
+  auto s_full = [&](int t) { return bar0 + 8u * (4 + 2 * NS + t); };    // S_t(j) ready
+  auto p_full = [&](int t) { return bar0 + 8u * (6 + 2 * NS + t); };    // P_t(j) written
+  auto o_full = [&](int t) { return bar0 + 8u * (8 + 2 * NS + t); };    // a unit's last P.V done
+  auto turn = [&](int t) { return bar0 + 8u * (10 + 2 * NS + t); };     // tile t may issue
+  const uint32_t drain = bar0 + 8u * (12 + 2 * NS);                     // every MMA done
   uint8_t* bar_ptr = smem + 2 * Cfg::kTileBytes + NS * Cfg::kTileBytes;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * Cfg::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- work unit: (batch*head, pair of query tiles)
-  const int BH = p.B * p.Hq;
-  int bh, unit;
-  if (p.lpt) {
-    unit = p.num_units - 1 - static_cast<int>(blockIdx.x) / BH;
-    bh = static_cast<int>(blockIdx.x) % BH;
-  } else {
-    unit = static_cast<int>(blockIdx.x) % p.num_units;
-    bh = static_cast<int>(blockIdx.x) / p.num_units;
-  }
-  const int b = bh / p.Hq;
-  const int hq = bh - b * p.Hq;
-  const int bhkv = b * p.Hkv + hq / p.group;
-  const int row0_0 = unit * 2 * kBlockM;
-  const int row0_1 = row0_0 + kBlockM;
-  const int n0 = kv_tiles_for(p, row0_0);
-  const int n1 = kv_tiles_for(p, row0_1);
-  const int n_max = max(n0, n1);
+  const int cta = static_cast<int>(blockIdx.x);
+  const int G = static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
       mbar_init(q_full(t), 1);
+      mbar_init(q_empty(t), 1);
       mbar_init(s_full(t), 1);
-      mbar_init(p_full(t, 0), 4);  // one arrive per softmax warp
-      mbar_init(p_full(t, 1), 4);
+      mbar_init(p_full(t), 4);  // one arrive per softmax warp
+      mbar_init(turn(t), 1);
       mbar_init(o_full(t), 1);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
+      mbar_init(kv_empty(s), 2);  // released by both MMA threads
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, 2);  // one commit per MMA thread
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -202,118 +238,152 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
     regs_decrease<kCtrlRegs>();
     if (warp == kLoadWarp) {
       // ------------------------------------------------------ TMA producer
+      // Per unit: K_0, V_0 through the ring, then Q_0, Q_1 (each once the
+      // previous unit's last S MMA on that buffer is done), then K_1, V_1, ...
+      // Loading K_0 and V_0 first lets them land while the previous unit
+      // finishes.
       if (lane == 0) {
         tma_prefetch_desc(&p.tm_q);
         tma_prefetch_desc(&p.tm_k);
         tma_prefetch_desc(&p.tm_v);
-        tma_prefetch_desc(&p.tm_o);
-        if (n0 > 0) {
-          mbar_arrive_expect_tx(q_full(0), Cfg::kTileBytes);
-          for (int blk = 0; blk < Cfg::kBlocks; ++blk)
-            tma_load_3d(sQ + blk * Cfg::kBlockBytes, &p.tm_q, blk * 64, row0_0, bh, q_full(0));
-        }
-        if (n1 > 0) {
-          mbar_arrive_expect_tx(q_full(1), Cfg::kTileBytes);
-          for (int blk = 0; blk < Cfg::kBlocks; ++blk)
-            tma_load_3d(sQ + Cfg::kTileBytes + blk * Cfg::kBlockBytes, &p.tm_q, blk * 64, row0_1, bh, q_full(1));
-        }
-        int issued = 0;
-        const int total = 2 * n_max;  // K_0, V_0, K_1, V_1, ...
+        int it = 0;  // K/V tiles issued so far (ring position)
+        int ui = 0;  // units started so far
+        bool ok = true;
+        // Q_0 and Q_1 of unit u, each once the previous unit's last S MMA on
+        // that buffer is done (a tile with no key tiles only completes the phase).
+        auto load_q = [&](const Unit& u) -> bool {
+          for (int t = 0; t < 2; ++t) {
+            if (ui > 0 && !mbar_wait(q_empty(t), (ui - 1) & 1, abort_flag)) return false;
+            if ((t ? u.n1 : u.n0) > 0) {
+              mbar_arrive_expect_tx(q_full(t), Cfg::kTileBytes);
+              for (int blk = 0; blk < Cfg::kBlocks; ++blk)
+                tma_load_3d(sQ + t * Cfg::kTileBytes + blk * Cfg::kBlockBytes, &p.tm_q, blk * 64,
+                            u.row0_0 + t * kBlockM, u.bh, q_full(t));
+            } else {
+              mbar_arrive(q_full(t));
+            }
+          }
+          return true;
+        };
 #pragma unroll 1
-        for (int it = 0; it < total; ++it) {
-          const int slot = it % NS;
-          if (!mbar_wait(kv_empty(slot), ((it / NS) & 1) ^ 1, abort_flag)) break;
-          mbar_arrive_expect_tx(kv_full(slot), Cfg::kTileBytes);
-          const CUtensorMap* tm = (it & 1) ? &p.tm_v : &p.tm_k;
-          const uint32_t dst = sKV + slot * Cfg::kTileBytes;
-          for (int blk = 0; blk < Cfg::kBlocks; ++blk)
-            tma_load_3d(dst + blk * Cfg::kBlockBytes, tm, blk * 64, (it >> 1) * kBlockN, bhkv, kv_full(slot));
-          ++issued;
+        for (int r = 0; ok; ++r) {
+          const int idx = unit_index(r, cta, G);
+          if (idx >= p.total_units) break;
+          const Unit u = make_unit(p, idx);
+          if (u.n_max <= 1) ok = load_q(u);
+#pragma unroll 1
+          for (int x = 0; ok && x < 2 * u.n_max; ++x, ++it) {  // K_0, V_0, K_1, V_1, ...
+            if (x == 2 && !load_q(u)) {  // this unit's Q after its K_0, V_0
+              ok = false;
+              break;
+            }
+            const int slot = it % NS;
+            if (!mbar_wait(kv_empty(slot), ((it / NS) & 1) ^ 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(kv_full(slot), Cfg::kTileBytes);
+            const CUtensorMap* tm = (x & 1) ? &p.tm_v : &p.tm_k;
+            const uint32_t dst = sKV + slot * Cfg::kTileBytes;
+            for (int blk = 0; blk < Cfg::kBlocks; ++blk)
+              tma_load_3d(dst + blk * Cfg::kBlockBytes, tm, blk * 64, (x >> 1) * kBlockN, u.bhkv, kv_full(slot));
+          }
+          ++ui;
         }
         // Copies still in flight must land before the CTA may exit.
-        if (n0 > 0) mbar_wait_drain(q_full(0), 0);
-        if (n1 > 0) mbar_wait_drain(q_full(1), 0);
-        for (int it = max(0, issued - NS); it < issued; ++it) mbar_wait_drain(kv_full(it % NS), (it / NS) & 1);
+        if (ui > 0) {
+          mbar_wait_drain(q_full(0), (ui - 1) & 1);
+          mbar_wait_drain(q_full(1), (ui - 1) & 1);
+        }
+        for (int i = max(0, it - NS); i < it; ++i) mbar_wait_drain(kv_full(i % NS), (i / NS) & 1);
       }
       __syncwarp();
-    } else if (warp == kMmaWarp) {
-      // --------------------------------------------------------- MMA issuer
+    } else if (warp == kMmaWarp || warp == kMmaWarp1) {
+      // ---------------------------------------------- MMA issuer of tile t
+      // Segment k of tile t in a unit is O_t += P_t(k-1) V_{k-1} (k >= 1)
+      // followed by S_t(k) = Q_t K_k^T (k < n_t): 16 MMAs, issued back to back
+      // once everything they read is ready.  The two issuers take turns (tile
+      // 0 segment k, tile 1 segment k, tile 0 segment k+1, ...) through the
+      // turn barriers, so the tensor core runs one tile's segment at a time --
+      // a tile's softmax waits for its own segment only -- while the other
+      // issuer's waits (for its P, its K/V slot, its turn) overlap the MMAs in
+      // flight.  Both issuers walk all n_max + 1 segments of every unit and
+      // release every K/V slot once, so kv_empty and turn see one arrival per
+      // phase from each.
+      const int t = (warp == kMmaWarp) ? 0 : 1;
       if (lane == 0) {
-        bool ok = true;
         const uint64_t hi = static_cast<uint64_t>(sdesc_hi(1024)) << 32;  // 8-row groups 1024 B apart
-        const uint64_t dq0 = hi | sdesc_lo(sQ, 16);
-        const uint64_t dq1 = hi | sdesc_lo(sQ + Cfg::kTileBytes, 16);
+        const uint64_t dq = hi | sdesc_lo(sQ + t * Cfg::kTileBytes, 16);
         auto dk = [&](int slot) { return hi | sdesc_lo(sKV + slot * Cfg::kTileBytes, 16); };
         auto dv = [&](int slot) { return hi | sdesc_lo(sKV + slot * Cfg::kTileBytes, Cfg::kBlockBytes); };
-        const uint32_t tS0 = tmem, tS1 = tmem + kBlockN;
-        const uint32_t tO0 = tmem + 2 * kBlockN, tO1 = tmem + 2 * kBlockN + D;
-        if (n0 > 0 && !mbar_wait(q_full(0), 0, abort_flag)) ok = false;
-        if (n1 > 0 && !mbar_wait(q_full(1), 0, abort_flag)) ok = false;
-        if (ok && n_max > 0) {
-          if (!mbar_wait(kv_full(0), 0, abort_flag)) {
-            ok = false;
-          } else {
-            tc_fence_after();
-            const uint64_t k0 = dk(0);
-            if (n0 > 0) {
-              issue_qk<D>(tS0, dq0, k0);
-              mma_commit(s_full(0));
-            }
-            if (n1 > 0) {
-              issue_qk<D>(tS1, dq1, k0);
-              mma_commit(s_full(1));
-            }
-            mma_commit(kv_empty(0));
-          }
-        }
+        const uint32_t tS = tmem + t * kBlockN;
+        const uint32_t tO = tmem + 2 * kBlockN + t * D;
+        int it_base = 0;  // ring position of the unit's K_0
+        int seg = 0;      // segments walked (the same count on both issuers)
+        int pj = 0;       // P_t tiles consumed (p_full phase)
+        int ui = 0;       // units walked (q_full phase)
+        bool ok = true;
 #pragma unroll 1
-        for (int j = 0; ok && j < n_max; ++j) {
-          const int itv = 2 * j + 1;
-          const int slot_v = itv % NS;
-          const int itk = 2 * j + 2;
-          const int slot_k = itk % NS;
-          if (!mbar_wait(kv_full(slot_v), (itv / NS) & 1, abort_flag)) break;
-          const uint64_t v_desc = dv(slot_v);
-          const uint64_t k_desc = dk(slot_k);
-          bool k_ready = false;
+        for (int r = 0; ok; ++r) {
+          const int idx = unit_index(r, cta, G);
+          if (idx >= p.total_units) break;
+          const Unit u = make_unit(p, idx);
+          const int nt = t ? u.n1 : u.n0;  // n0 <= n1: tile 1's rows come later
+          if (!mbar_wait(q_full(t), ui & 1, abort_flag)) break;
+          if (nt == 0) mma_commit(q_empty(t));  // nothing reads Q_t in this unit
 #pragma unroll 1
-          for (int t = 0; t < 2; ++t) {
-            const int nt = t ? n1 : n0;
-            if (j >= nt) continue;
-            const uint32_t tO = t ? tO1 : tO0;
-            const uint32_t tS = t ? tS1 : tS0;
-            // first half of P.V as soon as the softmax has written it
-            if (!mbar_wait(p_full(t, 0), j & 1, abort_flag)) {
-              ok = false;
-              break;
+          for (int k = 0; k <= u.n_max; ++k, ++seg) {
+            int slot_v = -1, slot_k = -1;
+            if (k >= 1) {
+              const int itv = it_base + 2 * k - 1;  // V_{k-1}
+              slot_v = itv % NS;
+              if (!mbar_wait(kv_full(slot_v), (itv / NS) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              if (k - 1 < nt && !mbar_wait(p_full(t), pj & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
             }
-            tc_fence_after();
-            issue_pv<D, 0>(tO, tS, v_desc, j > 0);
-            if (!mbar_wait(p_full(t, 1), j & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            issue_pv<D, 1>(tO, tS, v_desc, true);
-            const bool more = j + 1 < nt;
-            if (more && !k_ready) {
+            if (k < u.n_max) {
+              const int itk = it_base + 2 * k;  // K_k
+              slot_k = itk % NS;
               if (!mbar_wait(kv_full(slot_k), (itk / NS) & 1, abort_flag)) {
                 ok = false;
                 break;
               }
-              tc_fence_after();
-              k_ready = true;
             }
-            if (more) {
-              issue_qk<D>(tS, t ? dq1 : dq0, k_desc);
+            if (t == 1) {
+              if (!mbar_wait(turn(1), seg & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+            } else if (seg >= 1) {
+              if (!mbar_wait(turn(0), (seg - 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+            }
+            tc_fence_after();
+            if (k >= 1 && k - 1 < nt) {
+              const uint64_t v_desc = dv(slot_v);
+              issue_pv<D, 0>(tO, tS, v_desc, k > 1);
+              issue_pv<D, 1>(tO, tS, v_desc, true);
+              ++pj;
+              if (k == nt) mma_commit(o_full(t));
+            }
+            if (k < nt) {
+              issue_qk<D>(tS, dq, dk(slot_k));
               mma_commit(s_full(t));
-            } else {
-              mma_commit(o_full(t));
+              if (k == nt - 1) mma_commit(q_empty(t));
             }
+            if (slot_v >= 0) mma_commit(kv_empty(slot_v));
+            if (slot_k >= 0) mma_commit(kv_empty(slot_k));
+            mbar_arrive(turn(1 - t));
           }
-          if (!ok) break;
-          mma_commit(kv_empty(slot_v));
-          if (k_ready) mma_commit(kv_empty(slot_k));
+          it_base += 2 * u.n_max;
+          ++ui;
         }
         // Every MMA this thread issued must finish before TMEM is released.
         mma_commit(drain);
@@ -327,146 +397,154 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
     const int t = warp >> 2;      // query tile 0 or 1
     const int wq = warp & 3;      // TMEM lane quarter of this warp
     const int r_in_tile = wq * 32 + lane;
-    const int row0 = t ? row0_1 : row0_0;
-    const int row = row0 + r_in_tile;
-    const int n = t ? n1 : n0;
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_bits + t * kBlockN;
     const uint32_t tO = tmem + lane_bits + 2 * kBlockN + t * D;
     const float c = p.scale_log2;
-    const int row_limit = p.causal ? row + p.causal_offset : INT_MAX - kBlockN;
-    float m_used = -INFINITY;
-    float l = 0.f;
+    int sj = 0;  // S_t tiles consumed (s_full phase)
+    int ou = 0;  // units whose O_t was read (o_full phase)
     bool ok = true;
+#pragma unroll 1
+    for (int r = 0; ok; ++r) {
+      const int idx = unit_index(r, cta, G);
+      if (idx >= p.total_units) break;
+      const Unit u = make_unit(p, idx);
+      const int row0 = u.row0_0 + t * kBlockM;
+      const int row = row0 + r_in_tile;
+      const int n = t ? u.n1 : u.n0;
+      const int row_limit = p.causal ? row + p.causal_offset : INT_MAX - kBlockN;
+      float m_used = -INFINITY;
+      float l = 0.f;
 
 #pragma unroll 1
-    for (int j = 0; j < n; ++j) {
-      if (!mbar_wait(s_full(t), j & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t sv[128];
+      for (int j = 0; j < n; ++j, ++sj) {
+        if (!mbar_wait(s_full(t), sj & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sv[128];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[q * 32]));
-      tmem_wait_ld();
+        for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[q * 32]));
+        tmem_wait_ld();
 
-      const int k0 = j * kBlockN;
-      const bool need_mask = (k0 + kBlockN > p.Sk) || (p.causal && k0 + kBlockN - 1 > row0 + p.causal_offset);
-      if (need_mask) {
-        const int lim = min(p.Sk - 1, row_limit) - k0;  // last visible column
+        const int k0 = j * kBlockN;
+        const bool need_mask = (k0 + kBlockN > p.Sk) || (p.causal && k0 + kBlockN - 1 > row0 + p.causal_offset);
+        if (need_mask) {
+          const int lim = min(p.Sk - 1, row_limit) - k0;  // last visible column
 #pragma unroll
-        for (int e = 0; e < 128; ++e)
-          if (e > lim) sv[e] = __float_as_uint(-INFINITY);
-      }
-      // row max over the 128 scores: four independent chains of 3-input max
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+          for (int e = 0; e < 128; ++e)
+            if (e > lim) sv[e] = __float_as_uint(-INFINITY);
+        }
+        // row max over the 128 scores: four independent chains of 3-input max
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < 128; e += 8) {
-        mx0 = max3f(mx0, __uint_as_float(sv[e + 0]), __uint_as_float(sv[e + 1]));
-        mx1 = max3f(mx1, __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]));
-        mx2 = max3f(mx2, __uint_as_float(sv[e + 4]), __uint_as_float(sv[e + 5]));
-        mx3 = max3f(mx3, __uint_as_float(sv[e + 6]), __uint_as_float(sv[e + 7]));
-      }
-      const float m_new = max3f(m_used, max3f(mx0, mx1, mx2), mx3);
-      // (m_new - m_used) is NaN while both are -inf: no rescale then.
-      const bool rescale = (m_new - m_used) * c > kRescaleThreshold;
-      float alpha = 1.f;
-      if (rescale) {
-        alpha = ex2_approx((m_used - m_new) * c);
-        m_used = m_new;
-        l *= alpha;
-      }
-      // O holds P.V of earlier tiles; the S wait above implies they are done.
-      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-        const float2 a2 = make_float2(alpha, alpha);
+        for (int e = 0; e < 128; e += 8) {
+          mx0 = max3f(mx0, __uint_as_float(sv[e + 0]), __uint_as_float(sv[e + 1]));
+          mx1 = max3f(mx1, __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]));
+          mx2 = max3f(mx2, __uint_as_float(sv[e + 4]), __uint_as_float(sv[e + 5]));
+          mx3 = max3f(mx3, __uint_as_float(sv[e + 6]), __uint_as_float(sv[e + 7]));
+        }
+        const float m_new = max3f(m_used, max3f(mx0, mx1, mx2), mx3);
+        // (m_new - m_used) is NaN while both are -inf: no rescale then.
+        const bool rescale = (m_new - m_used) * c > kRescaleThreshold;
+        float alpha = 1.f;
+        if (rescale) {
+          alpha = ex2_approx((m_used - m_new) * c);
+          m_used = m_new;
+          l *= alpha;
+        }
+        // O holds P.V of this unit's earlier tiles; the S wait above implies
+        // they are done (S_t(j) is issued after P_t(j-1).V by the same thread).
+        if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+          const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll 1
-        for (int q = 0; q < D / 32; ++q) {
-          uint32_t o[32];
-          tmem_ld32(tO + q * 32, o);
-          tmem_wait_ld();
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t o[32];
+            tmem_ld32(tO + q * 32, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float2 r = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2);
-            o[e] = __float_as_uint(r.x);
-            o[e + 1] = __float_as_uint(r.y);
+            for (int e = 0; e < 32; e += 2) {
+              const float2 rr = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2);
+              o[e] = __float_as_uint(rr.x);
+              o[e + 1] = __float_as_uint(rr.y);
+            }
+            tmem_st32(tO + q * 32, o);
           }
-          tmem_st32(tO + q * 32, o);
         }
-      }
-      const float mc = (m_used == -INFINITY) ? 0.f : m_used * c;
-      const float2 c2 = make_float2(c, c);
-      const float2 nmc2 = make_float2(-mc, -mc);
-      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        const float mc = (m_used == -INFINITY) ? 0.f : m_used * c;
+        const float2 c2 = make_float2(c, c);
+        const float2 nmc2 = make_float2(-mc, -mc);
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 64; e += 4) {
-          const int i = half * 64 + e;
-          const float2 x0 = __ffma2_rn(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), c2, nmc2);
-          const float2 x1 =
-              __ffma2_rn(make_float2(__uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3])), c2, nmc2);
-          const float2 p0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
-          const float2 p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
-          acc0 = __fadd2_rn(acc0, p0);
-          acc1 = __fadd2_rn(acc1, p1);
-          pk[e / 2] = pack_bf16x2(p0.x, p0.y);
-          pk[e / 2 + 1] = pack_bf16x2(p1.x, p1.y);
+          for (int e = 0; e < 64; e += 4) {
+            const int i = half * 64 + e;
+            const float2 x0 = __ffma2_rn(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), c2, nmc2);
+            const float2 x1 =
+                __ffma2_rn(make_float2(__uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3])), c2, nmc2);
+            const float2 p0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+            const float2 p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+            acc0 = __fadd2_rn(acc0, p0);
+            acc1 = __fadd2_rn(acc1, p1);
+            pk[e / 2] = pack_bf16x2(p0.x, p0.y);
+            pk[e / 2 + 1] = pack_bf16x2(p1.x, p1.y);
+          }
+          tmem_st32(tS + half * 32, pk);
         }
-        tmem_st32(tS + half * 32, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full(t, half));
+        if (lane == 0) mbar_arrive(p_full(t));
+        l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
       }
-      l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
-    }
+      if (!ok) break;
 
-    // ---- epilogue: O / l -> bf16 -> swizzled smem (this tile's Q buffer) -> TMA store
-    if (row0 < p.Sq) {
-      if (ok && n > 0 && !mbar_wait(o_full(t), 0, abort_flag)) ok = false;
-      tc_fence_after();
-      // A row whose running max is still -inf saw no visible key: O = 0 and
-      // LSE = -inf.
-      const bool empty_row = (m_used == -INFINITY) || !(l > 0.f);
-      const float inv_l = empty_row ? 0.f : 1.f / l;
-      const uint32_t stage = sQ + t * Cfg::kTileBytes;
+      // ---- epilogue: O / l -> bf16 -> global (one thread per row)
+      if (row0 < p.Sq) {
+        if (n > 0) {
+          if (!mbar_wait(o_full(t), ou & 1, abort_flag)) ok = false;
+          ++ou;
+        }
+        tc_fence_after();
+        // A row whose running max is still -inf saw no visible key: O = 0 and
+        // LSE = -inf.
+        const bool empty_row = (m_used == -INFINITY) || !(l > 0.f);
+        const float inv_l = empty_row ? 0.f : 1.f / l;
+        uint16_t* dst = p.o + (static_cast<int64_t>(u.bh) * p.Sq + row) * D;
 #pragma unroll 1
-      for (int q = 0; q < D / 32; ++q) {
-        uint32_t o[32];
-        if (ok && n > 0) {
-          tmem_ld32(tO + q * 32, o);
-          tmem_wait_ld();
-        } else {
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t o[32];
+          if (ok && n > 0) {
+            tmem_ld32(tO + q * 32, o);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
-        }
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
+          }
+          if (row < p.Sq) {
 #pragma unroll
-        for (int c16 = 0; c16 < 4; ++c16) {
-          const int chunk = q * 4 + c16;  // 16-byte chunk index in the row (8 bf16 each)
-          const int blk = chunk >> 3;
-          const int cw = (chunk & 7) ^ (r_in_tile & 7);
-          const uint32_t addr = stage + blk * Cfg::kBlockBytes + r_in_tile * 128 + cw * 16;
-          const uint32_t* f = &o[c16 * 8];
-          st_shared_v4(addr,
-                       pack_bf16x2(__uint_as_float(f[0]) * inv_l, __uint_as_float(f[1]) * inv_l),
-                       pack_bf16x2(__uint_as_float(f[2]) * inv_l, __uint_as_float(f[3]) * inv_l),
-                       pack_bf16x2(__uint_as_float(f[4]) * inv_l, __uint_as_float(f[5]) * inv_l),
-                       pack_bf16x2(__uint_as_float(f[6]) * inv_l, __uint_as_float(f[7]) * inv_l));
+            for (int c8 = 0; c8 < 4; ++c8) {
+              const uint32_t* f = &o[c8 * 8];
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(f[0]) * inv_l, __uint_as_float(f[1]) * inv_l);
+              w.y = pack_bf16x2(__uint_as_float(f[2]) * inv_l, __uint_as_float(f[3]) * inv_l);
+              w.z = pack_bf16x2(__uint_as_float(f[4]) * inv_l, __uint_as_float(f[5]) * inv_l);
+              w.w = pack_bf16x2(__uint_as_float(f[6]) * inv_l, __uint_as_float(f[7]) * inv_l);
+              *reinterpret_cast<uint4*>(dst + q * 32 + c8 * 8) = w;
+            }
+          }
         }
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(1 + t, 128);
-      if (r_in_tile == 0) {
-        for (int blk = 0; blk < Cfg::kBlocks; ++blk)
-          tma_store_3d(&p.tm_o, stage + blk * Cfg::kBlockBytes, blk * 64, row0, bh);
-        bulk_commit_group();
-        bulk_wait_group0();
-      }
-      if (p.lse != nullptr && row < p.Sq) {
-        const float lse = empty_row ? -INFINITY : (m_used * p.scale + lg2_approx(l) * 0.69314718055994531f);
-        p.lse[static_cast<int64_t>(bh) * p.Sq + row] = lse;
+        if (p.lse != nullptr && row < p.Sq) {
+          const float lse = empty_row ? -INFINITY : (m_used * p.scale + lg2_approx(l) * 0.69314718055994531f);
+          p.lse[static_cast<int64_t>(u.bh) * p.Sq + row] = lse;
+        }
+        // O_t may be overwritten by the next unit's first P.V only after every
+        // warp of this group has read it: that P.V waits for this group's P of
+        // the next unit, which each warp writes after its own reads here.
+        tc_fence_before();
       }
     }
   }

@@ -289,8 +289,8 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   attn_status_t s = check_common(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
   if (s != ATTN_OK) return s;
   if (B == 0 || Sq == 0) return ATTN_OK;
-  int dev = 0;
-  if ((s = current_device(&dev, nullptr)) != ATTN_OK) return s;
+  int dev = 0, sms = 0;
+  if ((s = current_device(&dev, &sms)) != ATTN_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t rows = static_cast<int64_t>(B) * Hq * Sq;
   if (Sk == 0) return launch_fill_empty(o, lse, rows, d, st);
@@ -300,9 +300,9 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   std::memset(&prm, 0, sizeof(prm));
   if (!make_map(&prm.tm_q, q, d, Sq, static_cast<int64_t>(B) * Hq, kBlockM) ||
       !make_map(&prm.tm_k, k, d, Sk, static_cast<int64_t>(B) * Hkv, kBlockN) ||
-      !make_map(&prm.tm_v, v, d, Sk, static_cast<int64_t>(B) * Hkv, kBlockN) ||
-      !make_map(&prm.tm_o, o, d, Sq, static_cast<int64_t>(B) * Hq, kBlockM))
+      !make_map(&prm.tm_v, v, d, Sk, static_cast<int64_t>(B) * Hkv, kBlockN))
     return ATTN_ERR_CUDA;
+  prm.o = static_cast<uint16_t*>(o);
   prm.lse = lse;
   prm.B = B;
   prm.Hq = Hq;
@@ -316,8 +316,11 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   prm.lpt = causal != ATTN_CAUSAL_NONE ? 1 : 0;
   prm.scale = sc;
   prm.scale_log2 = sc * 1.4426950408889634f;
-  const int64_t grid = static_cast<int64_t>(B) * Hq * prm.num_units;
-  if (grid > INT_MAX) return ATTN_ERR_SHAPE;
+  const int64_t units = static_cast<int64_t>(B) * Hq * prm.num_units;
+  if (units > INT_MAX / 2) return ATTN_ERR_SHAPE;
+  prm.total_units = static_cast<int>(units);
+  // Persistent grid: one CTA per SM (the kernel's shared memory allows one).
+  const int64_t grid = std::min<int64_t>(units, sms);
   if (d == 128) return launch_prefill<128, kStagesD128>(prm, static_cast<int>(grid), dev, st);
   return launch_prefill<64, kStagesD64>(prm, static_cast<int>(grid), dev, st);
 }
