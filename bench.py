@@ -395,7 +395,7 @@ def main():
     achieved = flops_step * args.steps / (sum(sum(v) for v in per_shape_ms.values()) / 1e3) / 1e12
     big = HEADLINE[-1].name
     traffic = measured_traffic(big)
-    roofline = {"bound": "tensor", "kernel": "prefill_kernel<128,4>", "achieved": round(achieved, 1),
+    roofline = {"bound": "tensor", "kernel": "prefill_kernel<128,5>", "achieved": round(achieved, 1),
                 "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
                 "peak_kind": f"{peaks_kind} bf16 dense (burst)", "traffic": traffic,
                 "traffic_workload": big}
