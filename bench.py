@@ -290,6 +290,28 @@ class GpuDecode:
                                  out=self.o, lse=self.lse)
 
 
+class GpuDecodeVarlen(GpuDecode):
+    """The decode workload over caches whose valid length differs per batch
+    (seeded lengths in [1, capacity], held on the device)."""
+
+    def __init__(self, w, rank: int, copies: int = 3):
+        super().__init__(w, rank, copies)
+        self.lens = inputs.decode_lengths(w)
+        self.seqlens = torch.tensor(self.lens, dtype=torch.int32, device="cuda")
+
+    def run(self):
+        import scaled_dot_product_fa2_b200 as sdpa
+        k, v = self.kv[self.i % len(self.kv)]
+        self.i += 1
+        sdpa.attn_decode_splitkv_varlen(self.q, k, v, self.seqlens, causal=self.w.causal, scale=self.w.scale,
+                                        workspace=self.ws, out=self.o, lse=self.lse)
+
+    def valid_bytes(self):
+        w = self.w
+        kv = sum(2 * w.Hkv * L * w.d * 2 for L in self.lens)
+        return kv + 2 * w.B * w.Hq * w.Sq * w.d * 2 + w.B * w.Hq * w.Sq * 4
+
+
 def timed_calls(fns, flush, reps: int, warmup: int):
     """Per-call CUDA-event times (ms) on the current stream, L2 flushed before each call."""
     stream = torch.cuda.current_stream()
@@ -473,6 +495,18 @@ def measure_breakdown(flush, peak_tf, hbm_gbs, rank, reps: int = 10):
         out[w.name] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4),
                        "splits": int(s.ws.numel() // (w.B * w.Hq * w.Sq * (w.d + 2) * 4)),
                        "launches_per_call": 2}
+        del s
+    for w in inputs.DECODE:
+        s = GpuDecodeVarlen(w, rank)
+
+        def batch(s=s):
+            for _ in range(DECODE_BATCH):
+                s.run()
+
+        ms = statistics.median(timed_calls([batch], slack_only, reps, 2)[0]) / DECODE_BATCH
+        gbs = s.valid_bytes() / ms / 1e6
+        out[w.name + "_varlen"] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4),
+                                   "lengths": s.lens, "launches_per_call": 2}
         del s
     torch.cuda.empty_cache()
     return out

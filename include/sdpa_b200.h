@@ -68,8 +68,10 @@ typedef enum {
   ATTN_ERR_DEVICE_TIMEOUT = 9, /* a bounded wait inside a kernel gave up */
   ATTN_ERR_ARCH = 10,          /* the current device is not compute capability 10.0 */
   ATTN_ERR_SCALE = 11,         /* scale is negative, NaN or infinite */
-  ATTN_ERR_SCRATCH_LIMIT = 12  /* attn_decode_splitkv_static: problem needs more than
+  ATTN_ERR_SCRATCH_LIMIT = 12, /* attn_decode_splitkv_static: problem needs more than
                                   ATTN_STATIC_SCRATCH_BYTES of scratch */
+  ATTN_ERR_SEQLEN = 13         /* reported by attn_check_device_error: a per-batch key length read
+                                  on the device was outside [0, cache capacity] and was clamped */
 } attn_status_t;
 
 enum { ATTN_CAUSAL_NONE = 0, ATTN_CAUSAL_TOP_LEFT = 1, ATTN_CAUSAL_BOTTOM_RIGHT = 2 };
@@ -122,6 +124,34 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
                                   int num_splits, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Split-KV decode over a KV cache whose valid length differs per batch and
+ * lives in device memory ("[onnxruntime] WebGPU FlashAttention: kernel fusion
+ * and variable sequence length", section 1: the decode reads seqlen_k on the
+ * GPU, and the launch size must not depend on a host copy of it, or the two
+ * race).
+ *   k_cache, v_cache  [B, Hkv, Sk_capacity, d] bf16; for batch b only keys
+ *                     0 .. seqlens_k[b]-1 are read as keys (the rest of the
+ *                     capacity may hold anything)
+ *   seqlens_k         device int32 [B], 4-byte aligned; read by the kernels
+ *                     only, so it may be written by earlier work on `stream`
+ *                     (no host synchronisation is needed or performed).  A
+ *                     value outside [0, Sk_capacity] is clamped and makes
+ *                     attn_check_device_error() return ATTN_ERR_SEQLEN.
+ *   causal            as for attn_decode_splitkv, aligned to each batch's own
+ *                     length: with ATTN_CAUSAL_BOTTOM_RIGHT query row i of
+ *                     batch b sees key j iff j <= i + seqlens_k[b] - Sq.
+ * The grid, the split count and the workspace size depend only on
+ * Sk_capacity (attn_decode_workspace_size(B, Hq, Hkv, Sq, Sk_capacity, d,
+ * num_splits)); each batch's valid tiles are spread evenly over the splits on
+ * the device.  A batch with length 0 (or a row that sees no key) gets o = 0
+ * and lse = -inf.  Everything else is as for attn_decode_splitkv.
+ */
+attn_status_t attn_decode_splitkv_varlen(const void* q, const void* k_cache, const void* v_cache,
+                                         const int* seqlens_k, void* o, float* lse, int B, int Hq, int Hkv, int Sq,
+                                         int Sk_capacity, int d, float scale, int causal, int num_splits,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Split-KV decode that allocates nothing and takes no workspace -- for callers
  * that cannot obtain device memory themselves: a plug-in whose host framework
  * owns every device allocation and hands none out, or a service that fixes its
@@ -155,8 +185,9 @@ const char* attn_status_string(attn_status_t status);
 /*
  * Synchronizes `stream`, then reads and clears the device error word.
  * Returns ATTN_ERR_DEVICE_TIMEOUT if a kernel gave up on a bounded wait since
- * the last check, ATTN_ERR_CUDA if the synchronization itself failed, else
- * ATTN_OK.
+ * the last check, else ATTN_ERR_SEQLEN if attn_decode_splitkv_varlen had to
+ * clamp a key length, ATTN_ERR_CUDA if the synchronization itself failed,
+ * else ATTN_OK.
  */
 attn_status_t attn_check_device_error(void* stream);
 

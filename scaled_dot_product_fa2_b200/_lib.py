@@ -16,10 +16,12 @@ STATUS_NAMES = {
     0: "ATTN_OK", 1: "ATTN_ERR_NULL", 2: "ATTN_ERR_SHAPE", 3: "ATTN_ERR_GQA", 4: "ATTN_ERR_HEADDIM",
     5: "ATTN_ERR_ALIGN", 6: "ATTN_ERR_CAUSAL", 7: "ATTN_ERR_WORKSPACE", 8: "ATTN_ERR_CUDA",
     9: "ATTN_ERR_DEVICE_TIMEOUT", 10: "ATTN_ERR_ARCH", 11: "ATTN_ERR_SCALE", 12: "ATTN_ERR_SCRATCH_LIMIT",
+    13: "ATTN_ERR_SEQLEN",
 }
 STATIC_SCRATCH_BYTES = 16 << 20
 EXPORTS = ("attn_fwd", "attn_decode_num_splits", "attn_decode_workspace_size", "attn_decode_splitkv",
-           "attn_decode_splitkv_static", "attn_status_string", "attn_check_device_error", "attn_version")
+           "attn_decode_splitkv_varlen", "attn_decode_splitkv_static", "attn_status_string",
+           "attn_check_device_error", "attn_version")
 
 _lock = threading.Lock()
 _lib = None
@@ -46,6 +48,8 @@ def _declare(lib):
     lib.attn_decode_workspace_size.restype = SZ
     lib.attn_decode_splitkv.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, P, SZ, P]
     lib.attn_decode_splitkv.restype = I
+    lib.attn_decode_splitkv_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, P, SZ, P]
+    lib.attn_decode_splitkv_varlen.restype = I
     lib.attn_decode_splitkv_static.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, P]
     lib.attn_decode_splitkv_static.restype = I
     lib.attn_status_string.argtypes = [I]

@@ -30,10 +30,12 @@ struct DecodeParams {
   CUtensorMap tm_k;       // [B*Hkv][Sk][d] bf16, box {64, 64, 1}, 128-byte swizzle
   CUtensorMap tm_v;       // [B*Hkv][Sk][d]
   const uint16_t* q;      // [B, Hq, Sq, d] bf16 bits
+  const int* seqlens_k;   // [B] valid keys of each batch's cache (device), or nullptr: all Sk
   float* part_o;          // [B*Hq*Sq][nsplit][d]  locally normalised partial outputs
   float2* part_ml;        // [B*Hq*Sq][nsplit]     (local max of scale*q.k, local sum)
   int B, Hq, Hkv, Sq, Sk, group;
-  int causal, causal_offset;  // key j visible to row i iff j <= i + causal_offset (if causal)
+  int causal;             // 0 none, 1 top-left, 2 bottom-right
+  int causal_offset;      // key j visible to row i iff j <= i + causal_offset (if causal; fixed-length caches)
   int nsplit;             // splits per (batch, kv head)
   int tiles_per_split;    // 64-key tiles per split
   int row_groups;         // ceil(group*Sq / 16)
@@ -102,9 +104,22 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
   const int b = bhkv / p.Hkv;
   const int hkv = bhkv - b * p.Hkv;
   const int rows_total = p.group * p.Sq;  // query rows sharing this KV head
-  const int total_tiles = (p.Sk + kDecKeys - 1) / kDecKeys;
-  const int tile_begin = split * p.tiles_per_split;
-  const int tile_end = min(total_tiles, tile_begin + p.tiles_per_split);
+  // Valid keys of this batch's cache.  With per-batch lengths (read here, on
+  // the device, so the grid never depends on them) this batch's tiles are
+  // spread evenly over the splits, and the mask is aligned to its own length.
+  int L = p.Sk;
+  int tps = p.tiles_per_split;
+  int coff = p.causal_offset;
+  if (p.seqlens_k != nullptr) {
+    const int raw = __ldg(p.seqlens_k + b);
+    L = min(max(raw, 0), p.Sk);
+    if (raw != L && threadIdx.x == 0 && split == 0 && rg == 0 && hkv == 0) atomicOr(&g_error_word, kErrSeqlen);
+    tps = ((L + kDecKeys - 1) / kDecKeys + p.nsplit - 1) / p.nsplit;
+    coff = (p.causal == 2) ? L - p.Sq : 0;
+  }
+  const int total_tiles = (L + kDecKeys - 1) / kDecKeys;
+  const int tile_begin = split * tps;
+  const int tile_end = min(total_tiles, tile_begin + tps);
   const int ntiles = max(0, tile_end - tile_begin);
   // first flattened (b*Hq + hq)*Sq + i row of this KV head
   const int64_t row_base = (static_cast<int64_t>(b) * p.Hq + static_cast<int64_t>(hkv) * p.group) * p.Sq;
@@ -176,7 +191,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
   for (int h = 0; h < 2; ++h) {
     const int lr = rg * kDecRows + qr + 8 * h;  // local row = g*Sq + i
     const int i = lr % p.Sq;
-    lim[h] = p.causal ? min(p.Sk - 1, i + p.causal_offset) : p.Sk - 1;
+    lim[h] = p.causal ? min(L - 1, i + coff) : L - 1;
   }
 
   float o[D / 8][4];

@@ -14,10 +14,12 @@ namespace sdpa {
 
 // Device-side error word of the library (one per device; the library is a
 // single translation unit, so it is defined here).  Bit kErrWaitTimeout is set
-// when a bounded wait gives up.
+// when a bounded wait gives up; bit kErrSeqlen when a kernel had to clamp a
+// per-batch key length read from device memory.
 __device__ unsigned int g_error_word = 0;
 
 constexpr unsigned int kErrWaitTimeout = 1u;
+constexpr unsigned int kErrSeqlen = 2u;  // a per-batch key length was outside [0, cache capacity]
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -338,9 +338,9 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int d,
   return decode_ws_bytes(B, Hq, Sq, d, ns);
 }
 
-attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
-                                  int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale, int causal,
-                                  int num_splits, void* workspace, size_t workspace_bytes, void* stream) {
+static attn_status_t decode_impl(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k,
+                                 void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale,
+                                 int causal, int num_splits, void* workspace, size_t workspace_bytes, void* stream) {
   attn_status_t s = check_common(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
   if (s != ATTN_OK) return s;
   if (num_splits < 0) return ATTN_ERR_SHAPE;
@@ -369,6 +369,7 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
   float* part_o = static_cast<float*>(workspace);
   float2* part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + rows * ns * d * sizeof(float));
   prm.q = static_cast<const uint16_t*>(q);
+  prm.seqlens_k = seqlens_k;
   prm.part_o = part_o;
   prm.part_ml = part_ml;
   prm.B = B;
@@ -390,6 +391,25 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
   return launch_decode<64>(prm, static_cast<int>(grid), part_o, part_ml, o, lse, rows, dev, st);
 }
 
+attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                                  int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale, int causal,
+                                  int num_splits, void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_impl(q, k_cache, v_cache, nullptr, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal, num_splits,
+                     workspace, workspace_bytes, stream);
+}
+
+attn_status_t attn_decode_splitkv_varlen(const void* q, const void* k_cache, const void* v_cache,
+                                         const int* seqlens_k, void* o, float* lse, int B, int Hq, int Hkv, int Sq,
+                                         int Sk_capacity, int d, float scale, int causal, int num_splits,
+                                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (B > 0 && Sq > 0 && Sk_capacity > 0) {
+    if (seqlens_k == nullptr) return ATTN_ERR_NULL;
+    if (!aligned(seqlens_k, 4)) return ATTN_ERR_ALIGN;
+  }
+  return decode_impl(q, k_cache, v_cache, seqlens_k, o, lse, B, Hq, Hkv, Sq, Sk_capacity, d, scale, causal,
+                     num_splits, workspace, workspace_bytes, stream);
+}
+
 const char* attn_status_string(attn_status_t status) {
   switch (status) {
     case ATTN_OK: return "ok";
@@ -405,6 +425,7 @@ const char* attn_status_string(attn_status_t status) {
     case ATTN_ERR_ARCH: return "the current device is not sm_100 (B200)";
     case ATTN_ERR_SCALE: return "scale must be 0 (default) or finite and > 0";
     case ATTN_ERR_SCRATCH_LIMIT: return "problem needs more than the library's static decode scratch (16 MiB)";
+    case ATTN_ERR_SEQLEN: return "a per-batch key length was outside [0, cache capacity] (clamped)";
   }
   return "unknown status";
 }
@@ -416,7 +437,7 @@ attn_status_t attn_check_device_error(void* stream) {
   if (word != 0) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(sdpa::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
-    return ATTN_ERR_DEVICE_TIMEOUT;
+    return (word & sdpa::kErrWaitTimeout) ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_ERR_SEQLEN;
   }
   return ATTN_OK;
 }

@@ -101,3 +101,16 @@ def make_qkv(B: int, Hq: int, Hkv: int, Sq: int, Sk: int, d: int, seed: int,
 
 def workload_inputs(w: Workload, dtype: torch.dtype = torch.bfloat16):
     return make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Sk, w.d, w.seed, dtype)
+
+
+def decode_lengths(w: Workload) -> list[int]:
+    """Seeded per-batch valid cache lengths for the variable-length decode:
+    batch 0 uses the whole capacity w.Sk, batch 1 a single key, the others are
+    uniform in [1, w.Sk] from a CPU generator seeded with w.seed + 77."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(w.seed) + 77)
+    lens = torch.randint(1, w.Sk + 1, (w.B,), generator=g, dtype=torch.int64).tolist()
+    lens[0] = w.Sk
+    if w.B > 1:
+        lens[1] = 1
+    return [int(x) for x in lens]

@@ -116,6 +116,37 @@ def attn_decode_splitkv(q, k_cache, v_cache, causal: int = CAUSAL_BOTTOM_RIGHT, 
     return out, lse
 
 
+def attn_decode_splitkv_varlen(q, k_cache, v_cache, seqlens_k, causal: int = CAUSAL_BOTTOM_RIGHT,
+                               scale: float = 0.0, num_splits: int = 0, workspace=None, out=None, lse=None,
+                               return_lse: bool = True):
+    """Split-KV decode over caches with per-batch valid lengths (``attn_decode_splitkv_varlen``).
+
+    ``k_cache``/``v_cache`` are [B, Hkv, capacity, d]; ``seqlens_k`` is an int32
+    CUDA tensor [B] of valid keys per batch, read on the device only.
+    Returns (o, lse).
+    """
+    B, Hq, Hkv, Sq, Sk, d = _shapes(q, k_cache, v_cache)
+    if not isinstance(seqlens_k, torch.Tensor) or seqlens_k.dtype != torch.int32 or seqlens_k.dim() != 1:
+        raise TypeError("seqlens_k must be an int32 tensor [B]")
+    if tuple(seqlens_k.shape) != (B,) or seqlens_k.device != q.device or not seqlens_k.is_contiguous():
+        raise ValueError("seqlens_k must be a contiguous [B] tensor on q's device")
+    out, lse = _outputs(q, out, lse, return_lse)
+    if workspace is None:
+        workspace = decode_workspace(q, k_cache, num_splits)
+    if workspace.device != q.device or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous buffer on q's device")
+    lib = _lib.get()
+    with torch.cuda.device(q.device):
+        st = lib.attn_decode_splitkv_varlen(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                            seqlens_k.data_ptr(), out.data_ptr(),
+                                            lse.data_ptr() if lse is not None else None,
+                                            B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal), int(num_splits),
+                                            workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                            _stream_handle(q.device))
+    _lib.check(st, "attn_decode_splitkv_varlen")
+    return out, lse
+
+
 def attn_decode_splitkv_static(q, k_cache, v_cache, causal: int = CAUSAL_BOTTOM_RIGHT, scale: float = 0.0,
                                num_splits: int = 0, out=None, lse=None, return_lse: bool = True):
     """Split-KV decode without a workspace (``attn_decode_splitkv_static``).

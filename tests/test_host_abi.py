@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(12):
+    for code in range(14):
         assert lib.attn_status_string(code)
     assert lib.attn_status_string(0) == b"ok"
 
@@ -101,6 +101,18 @@ def test_decode_rejects_bad_workspace_on_host(lib):
     assert call(P, need - 1) == 7
     assert lib.attn_decode_splitkv(P, P, P, P, None, 2, 4, 2, 1, 256, 128, 0.0, 2, -1, P, need, None) == 2
     assert lib.attn_decode_splitkv(P, P, P, P, None, 2, 4, 3, 1, 256, 128, 0.0, 2, 0, P, need, None) == 3
+
+
+def test_varlen_decode_rejects_bad_lengths_pointer_on_host(lib):
+    args = (2, 4, 2, 1, 256, 128)
+    need = lib.attn_decode_workspace_size(*args, 0)
+    call = lambda seqlens: lib.attn_decode_splitkv_varlen(P, P, P, seqlens, P, None, *args, 0.0, 2, 0, P, need, None)
+    assert call(None) == 1      # ATTN_ERR_NULL
+    assert call(P + 2) == 5     # ATTN_ERR_ALIGN (int32 array)
+    # an empty problem needs no lengths
+    assert lib.attn_decode_splitkv_varlen(None, None, None, None, None, None, 0, 4, 2, 1, 256, 128, 0.0, 2, 0,
+                                          None, 0, None) == 0
+    assert lib.attn_status_string(13)
 
 
 def test_ptxas_report_checker():
