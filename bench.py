@@ -263,6 +263,24 @@ class GpuPrefill:
         return self.o.numel() * 2 + self.lse.numel() * 4
 
 
+class GpuPrefillVarlen(GpuPrefill):
+    """Causal prefill over padded sequences of seeded lengths (query and key
+    lengths equal per sequence); FLOPs count the valid causal work only."""
+
+    def __init__(self, w, rank: int):
+        super().__init__(w, rank)
+        self.lens = inputs.prefill_lengths(w)
+        self.seqlens = torch.tensor(self.lens, dtype=torch.int32, device="cuda")
+
+    def run(self):
+        import scaled_dot_product_fa2_b200 as sdpa
+        sdpa.attn_fwd_varlen(self.q, self.k, self.v, self.seqlens, self.seqlens, causal=self.w.causal,
+                             scale=self.w.scale, out=self.o, lse=self.lse)
+
+    def flops(self):
+        return sum(2.0 * self.w.Hq * L * L * self.w.d for L in self.lens)
+
+
 class GpuDecode:
     def __init__(self, w, rank: int, copies: int = 3):
         import scaled_dot_product_fa2_b200 as sdpa
@@ -474,6 +492,13 @@ def measure_breakdown(flush, peak_tf, hbm_gbs, rank, reps: int = 10):
         tf = w.flops() / ms / 1e9
         out[w.name] = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac": round(tf / peak_tf, 4)}
         del s
+    sv = GpuPrefillVarlen(inputs.PREFILL_VARLEN, rank)
+    ms = statistics.median(timed_calls([sv.run], flush, reps, 3)[0])
+    tf = sv.flops() / ms / 1e9
+    out[inputs.PREFILL_VARLEN.name] = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac": round(tf / peak_tf, 4),
+                                       "lengths": sv.lens}
+    del sv
+
     # Decode streams 268 MB per call from one of three rotating cache copies
     # (768 MiB > L2), so no call finds its K/V in L2.  No write flush here: a
     # flush leaves up to an L2's worth of dirty lines that the decode's reads

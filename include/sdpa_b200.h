@@ -70,8 +70,8 @@ typedef enum {
   ATTN_ERR_SCALE = 11,         /* scale is negative, NaN or infinite */
   ATTN_ERR_SCRATCH_LIMIT = 12, /* attn_decode_splitkv_static: problem needs more than
                                   ATTN_STATIC_SCRATCH_BYTES of scratch */
-  ATTN_ERR_SEQLEN = 13         /* reported by attn_check_device_error: a per-batch key length read
-                                  on the device was outside [0, cache capacity] and was clamped */
+  ATTN_ERR_SEQLEN = 13         /* reported by attn_check_device_error: a per-batch length read on
+                                  the device was outside its valid range and was clamped */
 } attn_status_t;
 
 enum { ATTN_CAUSAL_NONE = 0, ATTN_CAUSAL_TOP_LEFT = 1, ATTN_CAUSAL_BOTTOM_RIGHT = 2 };
@@ -84,6 +84,28 @@ enum { ATTN_CAUSAL_NONE = 0, ATTN_CAUSAL_TOP_LEFT = 1, ATTN_CAUSAL_BOTTOM_RIGHT 
  */
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                        int Sq, int Sk, int d, float scale, int causal, void* stream);
+
+/*
+ * Forward over a batch of sequences of different lengths, held padded:
+ *   q, o     [B, Hq,  Sq_max, d] bf16;  k, v [B, Hkv, Sk_max, d] bf16
+ *   seqlens_q, seqlens_k  device int32 [B], 4-byte aligned: batch b has
+ *            seqlens_q[b] query rows and seqlens_k[b] keys (the leading
+ *            rows of its padded tensors); read by the kernels only, so they
+ *            may be written by earlier work on `stream`.  A value outside
+ *            [0, Sq_max] resp. [0, Sk_max] is clamped and makes
+ *            attn_check_device_error() return ATTN_ERR_SEQLEN.
+ * Row i < seqlens_q[b] of batch b is attention over keys j < seqlens_k[b]
+ * with the mask aligned to the batch's own lengths (bottom-right: j <= i +
+ * seqlens_k[b] - seqlens_q[b]).  Padding rows (i >= seqlens_q[b]) of o and
+ * lse are not written, except when Sk_max == 0, where every row gets o = 0
+ * and lse = -inf.  The work list is built for Sq_max; units past a batch's
+ * length finish at once ("FlashAttention-2" notes, sequence-length
+ * parallelism; the variable-length decode input of the onnxruntime WebGPU
+ * page, section 1, applied to the forward pass).
+ */
+attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, const int* seqlens_q,
+                              const int* seqlens_k, void* o, float* lse, int B, int Hq, int Hkv, int Sq_max,
+                              int Sk_max, int d, float scale, int causal, void* stream);
 
 /*
  * Number of KV splits attn_decode_splitkv uses for this shape when called
@@ -185,9 +207,9 @@ const char* attn_status_string(attn_status_t status);
 /*
  * Synchronizes `stream`, then reads and clears the device error word.
  * Returns ATTN_ERR_DEVICE_TIMEOUT if a kernel gave up on a bounded wait since
- * the last check, else ATTN_ERR_SEQLEN if attn_decode_splitkv_varlen had to
- * clamp a key length, ATTN_ERR_CUDA if the synchronization itself failed,
- * else ATTN_OK.
+ * the last check, else ATTN_ERR_SEQLEN if attn_fwd_varlen or
+ * attn_decode_splitkv_varlen had to clamp a per-batch length, ATTN_ERR_CUDA
+ * if the synchronization itself failed, else ATTN_OK.
  */
 attn_status_t attn_check_device_error(void* stream);
 

@@ -19,7 +19,7 @@ STATUS_NAMES = {
     13: "ATTN_ERR_SEQLEN",
 }
 STATIC_SCRATCH_BYTES = 16 << 20
-EXPORTS = ("attn_fwd", "attn_decode_num_splits", "attn_decode_workspace_size", "attn_decode_splitkv",
+EXPORTS = ("attn_fwd", "attn_fwd_varlen", "attn_decode_num_splits", "attn_decode_workspace_size", "attn_decode_splitkv",
            "attn_decode_splitkv_varlen", "attn_decode_splitkv_static", "attn_status_string",
            "attn_check_device_error", "attn_version")
 
@@ -42,6 +42,8 @@ def _declare(lib):
     P, I, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.attn_fwd.restype = I
+    lib.attn_fwd_varlen.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.attn_fwd_varlen.restype = I
     lib.attn_decode_num_splits.argtypes = [I, I, I, I, I, I]
     lib.attn_decode_num_splits.restype = I
     lib.attn_decode_workspace_size.argtypes = [I, I, I, I, I, I, I]

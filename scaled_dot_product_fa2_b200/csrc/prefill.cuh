@@ -63,10 +63,12 @@ struct PrefillParams {
   CUtensorMap tm_v;  // [B*Hkv][Sk][d]
   uint16_t* o;       // [B*Hq][Sq][d] bf16 bits
   float* lse;        // [B*Hq*Sq] or nullptr
+  const int* seqlens_q;  // [B] valid query rows of each batch (device), or nullptr: all Sq
+  const int* seqlens_k;  // [B] valid keys of each batch (device), or nullptr: all Sk
   int B, Hq, Hkv, Sq, Sk;
   int group;          // Hq / Hkv
   int causal;         // 0 none, 1 top-left, 2 bottom-right
-  int causal_offset;  // key j visible to row i iff j <= i + causal_offset
+  int causal_offset;  // key j visible to row i iff j <= i + causal_offset (fixed lengths)
   int num_units;      // ceil(Sq / 256): work units per (batch, head)
   int total_units;    // B * Hq * num_units
   int lpt;            // 1: heaviest units first (causal)
@@ -98,13 +100,14 @@ struct PrefillCfg {
   static constexpr int kSmemBytes = (2 + NS) * kTileBytes + kNumBars * 8 + 16 + 1024;
 };
 
-// Number of 128-key tiles the query tile starting at row0 must visit.
-__device__ __forceinline__ int kv_tiles_for(const PrefillParams& p, int row0) {
-  if (row0 >= p.Sq || p.Sk <= 0) return 0;
-  int last_key = p.Sk - 1;
-  if (p.causal) {
-    const int last_row = min(row0 + kBlockM - 1, p.Sq - 1);
-    last_key = min(last_key, last_row + p.causal_offset);
+// Number of 128-key tiles the query tile starting at row0 must visit, for a
+// batch with Lq valid query rows, Lk valid keys and causal offset coff.
+__device__ __forceinline__ int kv_tiles_for(int causal, int Lq, int Lk, int coff, int row0) {
+  if (row0 >= Lq || Lk <= 0) return 0;
+  int last_key = Lk - 1;
+  if (causal) {
+    const int last_row = min(row0 + kBlockM - 1, Lq - 1);
+    last_key = min(last_key, last_row + coff);
   }
   if (last_key < 0) return 0;
   return last_key / kBlockN + 1;
@@ -128,7 +131,13 @@ __device__ __forceinline__ void unit_coords(const PrefillParams& p, int idx, int
 
 struct Unit {
   int bh, bhkv, row0_0, n0, n1, n_max;
+  int Lq, Lk, coff;  // this batch's valid query rows, valid keys, causal offset
 };
+
+// A per-batch length read from device memory, clamped to [0, cap].
+__device__ __forceinline__ int batch_length(const int* lens, int b, int cap) {
+  return lens == nullptr ? cap : min(max(__ldg(lens + b), 0), cap);
+}
 
 __device__ __forceinline__ Unit make_unit(const PrefillParams& p, int idx) {
   Unit u;
@@ -138,8 +147,12 @@ __device__ __forceinline__ Unit make_unit(const PrefillParams& p, int idx) {
   const int hq = u.bh - b * p.Hq;
   u.bhkv = b * p.Hkv + hq / p.group;
   u.row0_0 = v * 2 * kBlockM;
-  u.n0 = kv_tiles_for(p, u.row0_0);
-  u.n1 = kv_tiles_for(p, u.row0_0 + kBlockM);
+  u.Lq = batch_length(p.seqlens_q, b, p.Sq);
+  u.Lk = batch_length(p.seqlens_k, b, p.Sk);
+  u.coff = (p.seqlens_q == nullptr && p.seqlens_k == nullptr) ? p.causal_offset
+                                                               : (p.causal == 2 ? u.Lk - u.Lq : 0);
+  u.n0 = kv_tiles_for(p.causal, u.Lq, u.Lk, u.coff, u.row0_0);
+  u.n1 = kv_tiles_for(p.causal, u.Lq, u.Lk, u.coff, u.row0_0 + kBlockM);
   u.n_max = max(u.n0, u.n1);
   return u;
 }
@@ -270,6 +283,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
           const int idx = unit_index(r, cta, G);
           if (idx >= p.total_units) break;
           const Unit u = make_unit(p, idx);
+          if (p.seqlens_q != nullptr || p.seqlens_k != nullptr) {
+            const int b = u.bh / p.Hq;
+            const bool bad_q = p.seqlens_q != nullptr && __ldg(p.seqlens_q + b) != u.Lq;
+            const bool bad_k = p.seqlens_k != nullptr && __ldg(p.seqlens_k + b) != u.Lk;
+            if (bad_q || bad_k) atomicOr(&g_error_word, kErrSeqlen);
+          }
           if (u.n_max <= 1) ok = load_q(u);
 #pragma unroll 1
           for (int x = 0; ok && x < 2 * u.n_max; ++x, ++it) {  // K_0, V_0, K_1, V_1, ...
@@ -412,7 +431,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
       const int row0 = u.row0_0 + t * kBlockM;
       const int row = row0 + r_in_tile;
       const int n = t ? u.n1 : u.n0;
-      const int row_limit = p.causal ? row + p.causal_offset : INT_MAX - kBlockN;
+      const int row_limit = p.causal ? row + u.coff : INT_MAX - kBlockN;
       float m_used = -INFINITY;
       float l = 0.f;
 
@@ -429,9 +448,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
         tmem_wait_ld();
 
         const int k0 = j * kBlockN;
-        const bool need_mask = (k0 + kBlockN > p.Sk) || (p.causal && k0 + kBlockN - 1 > row0 + p.causal_offset);
+        const bool need_mask = (k0 + kBlockN > u.Lk) || (p.causal && k0 + kBlockN - 1 > row0 + u.coff);
         if (need_mask) {
-          const int lim = min(p.Sk - 1, row_limit) - k0;  // last visible column
+          const int lim = min(u.Lk - 1, row_limit) - k0;  // last visible column
 #pragma unroll
           for (int e = 0; e < 128; ++e)
             if (e > lim) sv[e] = __float_as_uint(-INFINITY);
@@ -503,7 +522,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
       if (!ok) break;
 
       // ---- epilogue: O / l -> bf16 -> global (one thread per row)
-      if (row0 < p.Sq) {
+      if (row0 < u.Lq) {
         if (n > 0) {
           if (!mbar_wait(o_full(t), ou & 1, abort_flag)) ok = false;
           ++ou;
@@ -524,7 +543,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = 0u;
           }
-          if (row < p.Sq) {
+          if (row < u.Lq) {
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8) {
               const uint32_t* f = &o[c8 * 8];
@@ -537,7 +556,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
             }
           }
         }
-        if (p.lse != nullptr && row < p.Sq) {
+        if (p.lse != nullptr && row < u.Lq) {
           const float lse = empty_row ? -INFINITY : (m_used * p.scale + lg2_approx(l) * 0.69314718055994531f);
           p.lse[static_cast<int64_t>(u.bh) * p.Sq + row] = lse;
         }

@@ -284,8 +284,9 @@ using namespace sdpa;
 
 extern "C" {
 
-attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                       int Sq, int Sk, int d, float scale, int causal, void* stream) {
+static attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int* seqlens_q,
+                              const int* seqlens_k, void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Sk,
+                              int d, float scale, int causal, void* stream) {
   attn_status_t s = check_common(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
   if (s != ATTN_OK) return s;
   if (B == 0 || Sq == 0) return ATTN_OK;
@@ -304,6 +305,8 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
     return ATTN_ERR_CUDA;
   prm.o = static_cast<uint16_t*>(o);
   prm.lse = lse;
+  prm.seqlens_q = seqlens_q;
+  prm.seqlens_k = seqlens_k;
   prm.B = B;
   prm.Hq = Hq;
   prm.Hkv = Hkv;
@@ -323,6 +326,21 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   const int64_t grid = std::min<int64_t>(units, sms);
   if (d == 128) return launch_prefill<128, kStagesD128>(prm, static_cast<int>(grid), dev, st);
   return launch_prefill<64, kStagesD64>(prm, static_cast<int>(grid), dev, st);
+}
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                       int Sq, int Sk, int d, float scale, int causal, void* stream) {
+  return fwd_impl(q, k, v, nullptr, nullptr, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal, stream);
+}
+
+attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, const int* seqlens_q,
+                              const int* seqlens_k, void* o, float* lse, int B, int Hq, int Hkv, int Sq_max,
+                              int Sk_max, int d, float scale, int causal, void* stream) {
+  if (B > 0 && Sq_max > 0) {
+    if (seqlens_q == nullptr || seqlens_k == nullptr) return ATTN_ERR_NULL;
+    if (!aligned(seqlens_q, 4) || !aligned(seqlens_k, 4)) return ATTN_ERR_ALIGN;
+  }
+  return fwd_impl(q, k, v, seqlens_q, seqlens_k, o, lse, B, Hq, Hkv, Sq_max, Sk_max, d, scale, causal, stream);
 }
 
 int attn_decode_num_splits(int B, int Hq, int Hkv, int Sq, int Sk, int d) {

@@ -114,3 +114,20 @@ def decode_lengths(w: Workload) -> list[int]:
     if w.B > 1:
         lens[1] = 1
     return [int(x) for x in lens]
+
+
+#: variable-length causal prefill: 8 sequences padded to 4096 (d=128, H=16),
+#: query and key lengths equal per sequence, drawn by ``prefill_lengths``
+PREFILL_VARLEN = Workload("prefill_varlen_causal_max4096", B=8, Hq=16, Hkv=16, Sq=4096, Sk=4096, d=128,
+                          causal=CAUSAL_TOP_LEFT, seed=6000)
+
+
+def prefill_lengths(w: Workload) -> list[int]:
+    """Seeded per-sequence lengths for the variable-length prefill: uniform in
+    [w.Sq // 8, w.Sq] from a CPU generator seeded with w.seed + 77; the first
+    sequence uses the full w.Sq."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(w.seed) + 77)
+    lens = torch.randint(w.Sq // 8, w.Sq + 1, (w.B,), generator=g, dtype=torch.int64).tolist()
+    lens[0] = w.Sq
+    return [int(x) for x in lens]

@@ -79,6 +79,36 @@ def attn_fwd(q, k, v, causal: int = CAUSAL_NONE, scale: float = 0.0, out=None, l
     return out, lse
 
 
+def _check_lengths(name, t, B, device):
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.int32 or t.dim() != 1:
+        raise TypeError(f"{name} must be an int32 tensor [B]")
+    if tuple(t.shape) != (B,) or t.device != device or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous [B] tensor on q's device")
+
+
+def attn_fwd_varlen(q, k, v, seqlens_q, seqlens_k, causal: int = CAUSAL_NONE, scale: float = 0.0, out=None,
+                    lse=None, return_lse: bool = True):
+    """Forward over padded sequences of per-batch lengths (``attn_fwd_varlen``).
+
+    q [B,Hq,Sq_max,d], k/v [B,Hkv,Sk_max,d]; ``seqlens_q``/``seqlens_k`` int32
+    CUDA tensors [B] read on the device.  Padding rows of the outputs are not
+    written (a new ``out`` is zero-filled so they read as 0).  Returns (o, lse).
+    """
+    B, Hq, Hkv, Sq, Sk, d = _shapes(q, k, v)
+    _check_lengths("seqlens_q", seqlens_q, B, q.device)
+    _check_lengths("seqlens_k", seqlens_k, B, q.device)
+    if out is None:
+        out = torch.zeros_like(q)
+    out, lse = _outputs(q, out, lse, return_lse)
+    lib = _lib.get()
+    with torch.cuda.device(q.device):
+        st = lib.attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), seqlens_q.data_ptr(),
+                                 seqlens_k.data_ptr(), out.data_ptr(), lse.data_ptr() if lse is not None else None,
+                                 B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal), _stream_handle(q.device))
+    _lib.check(st, "attn_fwd_varlen")
+    return out, lse
+
+
 def decode_num_splits(B, Hq, Hkv, Sq, Sk, d) -> int:
     return int(_lib.get().attn_decode_num_splits(B, Hq, Hkv, Sq, Sk, d))
 
@@ -126,10 +156,7 @@ def attn_decode_splitkv_varlen(q, k_cache, v_cache, seqlens_k, causal: int = CAU
     Returns (o, lse).
     """
     B, Hq, Hkv, Sq, Sk, d = _shapes(q, k_cache, v_cache)
-    if not isinstance(seqlens_k, torch.Tensor) or seqlens_k.dtype != torch.int32 or seqlens_k.dim() != 1:
-        raise TypeError("seqlens_k must be an int32 tensor [B]")
-    if tuple(seqlens_k.shape) != (B,) or seqlens_k.device != q.device or not seqlens_k.is_contiguous():
-        raise ValueError("seqlens_k must be a contiguous [B] tensor on q's device")
+    _check_lengths("seqlens_k", seqlens_k, B, q.device)
     out, lse = _outputs(q, out, lse, return_lse)
     if workspace is None:
         workspace = decode_workspace(q, k_cache, num_splits)

@@ -115,6 +115,15 @@ def test_varlen_decode_rejects_bad_lengths_pointer_on_host(lib):
     assert lib.attn_status_string(13)
 
 
+def test_varlen_forward_rejects_bad_lengths_pointers_on_host(lib):
+    call = lambda sq, sk: lib.attn_fwd_varlen(P, P, P, sq, sk, P, None, 2, 4, 2, 64, 64, 128, 0.0, 0, None)
+    assert call(None, P) == 1
+    assert call(P, None) == 1
+    assert call(P + 2, P) == 5
+    assert call(P, P + 1) == 5
+    assert lib.attn_fwd_varlen(None, None, None, None, None, None, None, 0, 4, 2, 64, 64, 128, 0.0, 0, None) == 0
+
+
 def test_ptxas_report_checker():
     regs = build.PREFILL_LAUNCH_REGS
     ok = ("ptxas info    : Compiling entry function '_ZN4sdpa14prefill_kernelILi128ELi4EEEvNS_13PrefillParamsE'\n"
