@@ -17,6 +17,9 @@ Sources followed (page title and section):
   * "[onnxruntime] WebGPU FlashAttention: kernel fusion ...", section 1
     (fused decode partial with (max, sum) metadata, VxReduce rescale)
       -> split_partials, split_combine
+  * same page, same section: additive attention bias applied with the causal
+    mask, two leading dims broadcasting over batch and heads
+      -> attn_fwd(..., bias=...), attn_rows(..., bias=...)
 """
 from __future__ import annotations
 
@@ -58,11 +61,15 @@ def bind(lib):
     lib.oracle_attn_fwd.argtypes = [_D, _D, _D, _D, _D, i, i, i, i, i, i, d, i, i]
     lib.oracle_attn_rows.argtypes = [_D, _D, _D, i, i, i, i, i, i, d, i,
                                      _I64, ctypes.c_int64, _D, _D, i]
+    lib.oracle_attn_fwd_bias.argtypes = [_D, _D, _D, _D, i, i, _D, _D, i, i, i, i, i, i, d, i, i]
+    lib.oracle_attn_rows_bias.argtypes = [_D, _D, _D, _D, i, i, i, i, i, i, i, i, d, i,
+                                          _I64, ctypes.c_int64, _D, _D, i]
     lib.oracle_online_attn.argtypes = [_D, _D, _D, _D, _D, i, i, i, i, i, i, d, i, i, i]
     lib.oracle_split_partials.argtypes = [_D, _D, _D, i, i, i, i, i, i, d, i,
                                           _I32, i, _D, _D, _D]
     lib.oracle_split_combine.argtypes = [_D, _D, _D, ctypes.c_int64, i, i, _D, _D]
-    for f in (lib.oracle_attn_fwd, lib.oracle_attn_rows, lib.oracle_online_attn,
+    for f in (lib.oracle_attn_fwd, lib.oracle_attn_rows, lib.oracle_attn_fwd_bias, lib.oracle_attn_rows_bias,
+              lib.oracle_online_attn,
               lib.oracle_split_partials, lib.oracle_split_combine):
         f.restype = ctypes.c_int
     return lib
@@ -99,21 +106,37 @@ def _threads(nthreads):
     return int(nthreads) if nthreads else (os.cpu_count() or 1)
 
 
-def attn_fwd(q, k, v, scale: float, causal: int = CAUSAL_NONE, nthreads: int | None = None):
-    """The five naive steps for every row.  Returns (o[B,Hq,Sq,d], lse[B,Hq,Sq])."""
+def _bias(bias, B, Hq, Sq, Sk):
+    """The bias as a contiguous fp64 [bias_b, bias_h, Sq, Sk] array and its two
+    broadcast dims (each 1 or the full size)."""
+    b = _f64(bias)
+    if b.ndim != 4 or b.shape[2:] != (Sq, Sk) or b.shape[0] not in (1, B) or b.shape[1] not in (1, Hq):
+        raise ValueError(f"bias must be [1|B, 1|Hq, Sq, Sk], got {b.shape}")
+    return b, int(b.shape[0]), int(b.shape[1])
+
+
+def attn_fwd(q, k, v, scale: float, causal: int = CAUSAL_NONE, nthreads: int | None = None, bias=None):
+    """The five naive steps for every row (the bias, if given, is added to the
+    scaled scores before the mask).  Returns (o[B,Hq,Sq,d], lse[B,Hq,Sq])."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, Hq, Hkv, Sq, Sk, d = _dims(q, k, v)
     o = np.zeros((B, Hq, Sq, d))
     lse = np.zeros((B, Hq, Sq))
-    st = _load().oracle_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                                 B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal),
-                                 _threads(nthreads))
+    if bias is None:
+        st = _load().oracle_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                     B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal),
+                                     _threads(nthreads))
+    else:
+        bb, nb, nh = _bias(bias, B, Hq, Sq, Sk)
+        st = _load().oracle_attn_fwd_bias(_ptr(q), _ptr(k), _ptr(v), _ptr(bb), nb, nh, _ptr(o), _ptr(lse),
+                                          B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal),
+                                          _threads(nthreads))
     if st != 0:
         raise ValueError(f"oracle_attn_fwd failed ({st})")
     return o, lse
 
 
-def attn_rows(q, k, v, scale: float, causal: int, rows, nthreads: int | None = None):
+def attn_rows(q, k, v, scale: float, causal: int, rows, nthreads: int | None = None, bias=None):
     """The five naive steps for selected rows.
 
     ``rows`` are flattened indices (b*Hq + hq)*Sq + i.  Returns (o[n,d], lse[n]).
@@ -124,9 +147,15 @@ def attn_rows(q, k, v, scale: float, causal: int, rows, nthreads: int | None = N
     n = rows.shape[0]
     o = np.zeros((n, d))
     lse = np.zeros((n,))
-    st = _load().oracle_attn_rows(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Sq, Sk, d,
-                                  float(scale), int(causal), rows.ctypes.data_as(_I64), n,
-                                  _ptr(o), _ptr(lse), _threads(nthreads))
+    if bias is None:
+        st = _load().oracle_attn_rows(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Sq, Sk, d,
+                                      float(scale), int(causal), rows.ctypes.data_as(_I64), n,
+                                      _ptr(o), _ptr(lse), _threads(nthreads))
+    else:
+        bb, nb, nh = _bias(bias, B, Hq, Sq, Sk)
+        st = _load().oracle_attn_rows_bias(_ptr(q), _ptr(k), _ptr(v), _ptr(bb), nb, nh, B, Hq, Hkv, Sq, Sk, d,
+                                           float(scale), int(causal), rows.ctypes.data_as(_I64), n,
+                                           _ptr(o), _ptr(lse), _threads(nthreads))
     if st != 0:
         raise ValueError(f"oracle_attn_rows failed ({st})")
     return o, lse

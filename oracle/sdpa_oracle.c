@@ -22,8 +22,16 @@
  *    locally normalised partial output per KV split plus (local max, local
  *    sum) metadata, and the reduce step rescales each partial so the result
  *    equals full softmax.V.  oracle_split_partials / oracle_split_combine.
+ *  - same page, same section: the fused decode kernel applies an optional
+ *    additive attention bias to the scores together with the causal mask; the
+ *    bias has two leading dimensions that broadcast over batch and heads
+ *    (attn_bias_dim0 / attn_bias_dim1, 1 when absent).  oracle_attn_fwd_bias /
+ *    oracle_attn_rows_bias.
  *
  * Readings (where the pages are silent):
+ *  - Bias: shape [bias_b, bias_h, Sq, Sk] with bias_b in {1, B} and bias_h in
+ *    {1, Hq} (1 = broadcast); it is added to the *scaled* scores, before the
+ *    mask: x_ij = scale * q.k + bias[b', h', i, j].  LSE is over these x.
  *  - LSE is the natural log of the softmax denominator over *scaled* scores:
  *    lse = max_j x_j + log(sum_j exp(x_j - max)), x = scale * q.k.
  *  - Causal alignment: mode 1 (top-left) keeps key j for query i iff j <= i;
@@ -49,6 +57,8 @@ typedef struct {
     int B, Hq, Hkv, Sq, Sk, d;
     double scale;
     int causal;
+    const double *bias; /* [bias_b, bias_h, Sq, Sk] or NULL */
+    int bias_b, bias_h;
 } attn_args;
 
 /* Is key j visible to query i?  (masked_fill step of the naive definition) */
@@ -77,8 +87,13 @@ static void attn_one_row(const attn_args *a, int b, int hq, int i,
         for (int c = 0; c < d; ++c) s += qrow[c] * kbase[(size_t)j * d + c];
         scores[j] = s;
     }
-    /* step 2: scores * scale */
+    /* step 2: scores * scale (+ the additive bias, if any) */
     for (int j = 0; j < Sk; ++j) scores[j] *= a->scale;
+    if (a->bias) {
+        const int bb = a->bias_b == 1 ? 0 : b, bh = a->bias_h == 1 ? 0 : hq;
+        const double *brow = a->bias + (((size_t)bb * a->bias_h + bh) * a->Sq + i) * (size_t)Sk;
+        for (int j = 0; j < Sk; ++j) scores[j] += brow[j];
+    }
     /* step 3: masked_fill(mask, -inf) */
     for (int j = 0; j < Sk; ++j)
         if (!key_visible(a->causal, i, j, a->Sq, Sk)) scores[j] = -INFINITY;
@@ -187,10 +202,26 @@ int oracle_attn_fwd(const double *q, const double *k, const double *v, double *o
         lse_buf = (double *)malloc(sizeof(double) * (size_t)(nrows > 0 ? nrows : 1));
         if (!lse_buf) return -2;
     }
-    attn_args a = {q, k, v, o, lse_buf, B, Hq, Hkv, Sq, Sk, d, scale, causal};
+    attn_args a = {q, k, v, o, lse_buf, B, Hq, Hkv, Sq, Sk, d, scale, causal, NULL, 1, 1};
     int st = run_rows(&a, NULL, nrows, o, lse_buf, nthreads);
     if (!lse) free(lse_buf);
     return st;
+}
+
+static int check_bias(int B, int Hq, int bias_b, int bias_h) {
+    if (!(bias_b == 1 || bias_b == B) || !(bias_h == 1 || bias_h == Hq)) return -1;
+    return 0;
+}
+
+/* oracle_attn_fwd with an additive bias [bias_b, bias_h, Sq, Sk]. */
+int oracle_attn_fwd_bias(const double *q, const double *k, const double *v, const double *bias,
+                         int bias_b, int bias_h, double *o, double *lse,
+                         int B, int Hq, int Hkv, int Sq, int Sk, int d, double scale, int causal,
+                         int nthreads) {
+    if (check_shape(B, Hq, Hkv, Sq, Sk, d, causal) || !bias || check_bias(B, Hq, bias_b, bias_h)) return -1;
+    if (!lse) return -1;
+    attn_args a = {q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal, bias, bias_b, bias_h};
+    return run_rows(&a, NULL, (int64_t)B * Hq * Sq, o, lse, nthreads);
 }
 
 /* Selected rows only: rows[n] are flattened (b*Hq + hq)*Sq + i indices;
@@ -203,7 +234,21 @@ int oracle_attn_rows(const double *q, const double *k, const double *v,
     const int64_t total = (int64_t)B * Hq * Sq;
     for (int64_t r = 0; r < n; ++r)
         if (rows[r] < 0 || rows[r] >= total) return -1;
-    attn_args a = {q, k, v, NULL, NULL, B, Hq, Hkv, Sq, Sk, d, scale, causal};
+    attn_args a = {q, k, v, NULL, NULL, B, Hq, Hkv, Sq, Sk, d, scale, causal, NULL, 1, 1};
+    return run_rows(&a, rows, n, o_rows, lse_rows, nthreads);
+}
+
+/* oracle_attn_rows with an additive bias [bias_b, bias_h, Sq, Sk]. */
+int oracle_attn_rows_bias(const double *q, const double *k, const double *v, const double *bias,
+                          int bias_b, int bias_h,
+                          int B, int Hq, int Hkv, int Sq, int Sk, int d, double scale, int causal,
+                          const int64_t *rows, int64_t n, double *o_rows, double *lse_rows,
+                          int nthreads) {
+    if (check_shape(B, Hq, Hkv, Sq, Sk, d, causal) || !bias || check_bias(B, Hq, bias_b, bias_h)) return -1;
+    const int64_t total = (int64_t)B * Hq * Sq;
+    for (int64_t r = 0; r < n; ++r)
+        if (rows[r] < 0 || rows[r] >= total) return -1;
+    attn_args a = {q, k, v, NULL, NULL, B, Hq, Hkv, Sq, Sk, d, scale, causal, bias, bias_b, bias_h};
     return run_rows(&a, rows, n, o_rows, lse_rows, nthreads);
 }
 

@@ -305,3 +305,104 @@ def test_partials_are_locally_normalised(oracle_mod):
     o_a, l_a = oracle_mod.attn_fwd(q, k[:, :, :4], v[:, :, :4], 0.5, NONE)
     np.testing.assert_allclose(po[0, 0, 0, 0], o_a[0, 0, 0], rtol=0, atol=1e-12)
     np.testing.assert_allclose(pm[0, 0, 0, 0] + math.log(pl[0, 0, 0, 0]), l_a[0, 0, 0], atol=1e-12)
+
+
+# --------------------------------------------------------------- additive bias
+# ("[onnxruntime] WebGPU FlashAttention: kernel fusion ...", section 1: the
+# fused decode applies an attention bias with the mask; its two leading dims
+# broadcast over batch and heads.)
+
+def brute_force_bias(q, k, v, bias, scale, causal):
+    """Independent scalar attention with an additive bias on the scaled scores."""
+    B, Hq, Sq, d = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    o = np.zeros((B, Hq, Sq, d))
+    lse = np.zeros((B, Hq, Sq))
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // G
+            bb, bh = (0 if bias.shape[0] == 1 else b), (0 if bias.shape[1] == 1 else h)
+            for i in range(Sq):
+                w = []
+                for j in range(Sk):
+                    if not _visible(causal, i, j, Sq, Sk):
+                        continue
+                    x = scale * math.fsum(float(q[b, h, i, c]) * float(k[b, hk, j, c]) for c in range(d))
+                    w.append((j, math.exp(x + float(bias[bb, bh, i, j]))))
+                w = [(j, e) for j, e in w if e > 0.0]
+                if not w:
+                    lse[b, h, i] = -math.inf
+                    continue
+                z = math.fsum(e for _, e in w)
+                lse[b, h, i] = math.log(z)
+                for c in range(d):
+                    o[b, h, i, c] = math.fsum(e * float(v[b, hk, j, c]) for j, e in w) / z
+    return o, lse
+
+
+@pytest.mark.parametrize("dims", [(1, 1), (2, 1), (1, 4), (2, 4)])
+@pytest.mark.parametrize("causal", [NONE, TL, BR])
+def test_bias_brute_force_every_broadcast(oracle_mod, dims, causal):
+    B, Hq, Hkv, Sq, Sk, d = 2, 4, 2, 3, 5, 3
+    q, k, v = _rand((B, Hq, Sq, d), 1), _rand((B, Hkv, Sk, d), 2), _rand((B, Hkv, Sk, d), 3)
+    bias = _rand((dims[0], dims[1], Sq, Sk), 4)
+    o, lse = oracle_mod.attn_fwd(q, k, v, 0.7, causal, bias=bias)
+    o_bf, lse_bf = brute_force_bias(q, k, v, bias, 0.7, causal)
+    assert np.allclose(o, o_bf, atol=1e-12, rtol=0)
+    assert np.allclose(lse, lse_bf, atol=1e-12, rtol=0)
+
+
+def test_bias_of_log_weights_with_zero_query_is_weighted_mean(oracle_mod):
+    """q = 0 makes every score 0, so bias_j = log w_j gives softmax weights
+    w_j / sum w: o = sum_j w_j v_j / sum_j w_j and lse = log sum_j w_j (a closed
+    form; a bias that were subtracted, scaled or applied after the softmax
+    fails it)."""
+    B, H, Sq, Sk, d = 1, 2, 3, 6, 4
+    q = np.zeros((B, H, Sq, d))
+    k, v = _rand((B, H, Sk, d), 5), _rand((B, H, Sk, d), 6)
+    w = np.random.default_rng(7).uniform(0.1, 3.0, size=(B, H, Sq, Sk))
+    o, lse = oracle_mod.attn_fwd(q, k, v, 0.9, NONE, bias=np.log(w))
+    expect = np.einsum("bhij,bhjc->bhic", w, v) / w.sum(-1, keepdims=True)
+    assert np.allclose(o, expect, atol=1e-12)
+    assert np.allclose(lse, np.log(w.sum(-1)), atol=1e-12)
+
+
+def test_constant_bias_per_row_shifts_lse_only(oracle_mod):
+    """Adding c_i to every score of row i leaves the softmax unchanged and adds
+    c_i to the row's LSE."""
+    B, Hq, Hkv, Sq, Sk, d = 1, 2, 1, 4, 9, 5
+    q, k, v = _rand((B, Hq, Sq, d), 8), _rand((B, Hkv, Sk, d), 9), _rand((B, Hkv, Sk, d), 10)
+    c = _rand((1, Hq, Sq, 1), 11) * 5.0
+    for causal in (NONE, BR):
+        o0, l0 = oracle_mod.attn_fwd(q, k, v, 0.4, causal)
+        o1, l1 = oracle_mod.attn_fwd(q, k, v, 0.4, causal, bias=np.broadcast_to(c, (1, Hq, Sq, Sk)))
+        assert np.allclose(o1, o0, atol=1e-12)
+        assert np.allclose(l1, l0 + c[..., 0], atol=1e-12)
+
+
+def test_minus_infinity_bias_masks_keys(oracle_mod):
+    """A -inf bias on a key is the same as removing that key; a row whose keys
+    are all -inf gives o = 0 and lse = -inf."""
+    B, H, Sq, Sk, d = 1, 1, 3, 6, 4
+    q, k, v = _rand((B, H, Sq, d), 12), _rand((B, H, Sk, d), 13), _rand((B, H, Sk, d), 14)
+    keep = np.array([0, 2, 5])
+    bias = np.full((1, 1, Sq, Sk), -np.inf)
+    bias[..., keep] = 0.0
+    bias[0, 0, 2, :] = -np.inf
+    o, lse = oracle_mod.attn_fwd(q, k, v, 0.6, NONE, bias=bias)
+    o_ref, lse_ref = oracle_mod.attn_fwd(q[:, :, :2], k[:, :, keep], v[:, :, keep], 0.6, NONE)
+    assert np.allclose(o[:, :, :2], o_ref, atol=1e-12)
+    assert np.allclose(lse[:, :, :2], lse_ref, atol=1e-12)
+    assert np.all(o[0, 0, 2] == 0.0) and lse[0, 0, 2] == -np.inf
+
+
+def test_bias_rows_api_matches_full(oracle_mod):
+    B, Hq, Hkv, Sq, Sk, d = 2, 2, 1, 5, 7, 3
+    q, k, v = _rand((B, Hq, Sq, d), 15), _rand((B, Hkv, Sk, d), 16), _rand((B, Hkv, Sk, d), 17)
+    bias = _rand((B, 1, Sq, Sk), 18)
+    o, lse = oracle_mod.attn_fwd(q, k, v, 0.5, TL, bias=bias)
+    rows = np.array([0, 3, 7, 12, 19])
+    o_r, l_r = oracle_mod.attn_rows(q, k, v, 0.5, TL, rows, bias=bias)
+    assert np.allclose(o_r, o.reshape(-1, d)[rows], atol=1e-13)
+    assert np.allclose(l_r, lse.reshape(-1)[rows], atol=1e-13)

@@ -29,6 +29,13 @@ MUTATIONS = {
     "combine_drops_local_sum": ("const double w = ls * exp(part_m[r * ns + s] - M);",
                                 "const double w = exp(part_m[r * ns + s] - M);"),
     "partials_not_local_max": ("const double p = exp(x[j] - mx);", "const double p = exp(x[j]);"),
+    "bias_subtracted": ("for (int j = 0; j < Sk; ++j) scores[j] += brow[j];",
+                        "for (int j = 0; j < Sk; ++j) scores[j] -= brow[j];"),
+    "bias_scaled": ("for (int j = 0; j < Sk; ++j) scores[j] += brow[j];",
+                    "for (int j = 0; j < Sk; ++j) scores[j] += a->scale * brow[j];"),
+    "bias_broadcast_swapped": ("const int bb = a->bias_b == 1 ? 0 : b, bh = a->bias_h == 1 ? 0 : hq;",
+                               "const int bb = a->bias_h == 1 ? 0 : b, bh = a->bias_b == 1 ? 0 : hq;"),
+    "bias_row_index": ("* a->Sq + i) * (size_t)Sk;", "* a->Sq + (a->Sq - 1 - i)) * (size_t)Sk;"),
 }
 
 
@@ -45,6 +52,9 @@ def _pin_suite(mod):
             pins.test_split_combine_equals_unsplit(mod, ns, causal)
     pins.test_split_with_masked_and_empty_splits(mod)
     pins.test_partials_are_locally_normalised(mod)
+    for dims in ((1, 1), (2, 1), (1, 4), (2, 4)):
+        pins.test_bias_brute_force_every_broadcast(mod, dims, 1)
+    pins.test_bias_of_log_weights_with_zero_query_is_weighted_mean(mod)
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
