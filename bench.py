@@ -492,6 +492,24 @@ def measure_breakdown(flush, peak_tf, hbm_gbs, rank, reps: int = 10):
         tf = w.flops() / ms / 1e9
         out[w.name] = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac": round(tf / peak_tf, 4)}
         del s
+    # the non-causal seq-2048 shape with an additive bias shared by all heads
+    # and batches ([1, 1, S, S] bf16, 8 MiB: it stays in L2, so this measures
+    # the bias path's compute cost)
+    wb = inputs.BY_NAME["prefill_noncausal_s2048"]
+    sb = GpuPrefill(wb, rank)
+    gb = torch.Generator().manual_seed(wb.seed + 99)
+    bias = torch.randn((1, 1, wb.Sq, wb.Sk), generator=gb).bfloat16().cuda()
+
+    def run_bias(sb=sb, bias=bias):
+        import scaled_dot_product_fa2_b200 as sdpa
+        sdpa.attn_fwd(sb.q, sb.k, sb.v, causal=wb.causal, scale=wb.scale, out=sb.o, lse=sb.lse, bias=bias)
+
+    ms = statistics.median(timed_calls([run_bias], flush, reps, 3)[0])
+    tf = wb.flops() / ms / 1e9
+    out[wb.name + "_bias"] = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac": round(tf / peak_tf, 4),
+                              "bias": "[1, 1, S, S] bf16"}
+    del sb, bias
+
     sv = GpuPrefillVarlen(inputs.PREFILL_VARLEN, rank)
     ms = statistics.median(timed_calls([sv.run], flush, reps, 3)[0])
     tf = sv.flops() / ms / 1e9

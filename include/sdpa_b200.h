@@ -77,6 +77,34 @@ typedef enum {
 enum { ATTN_CAUSAL_NONE = 0, ATTN_CAUSAL_TOP_LEFT = 1, ATTN_CAUSAL_BOTTOM_RIGHT = 2 };
 
 /*
+ * Optional inputs of attn_fwd_ex and attn_decode_splitkv_ex.  Zero-initialise
+ * (memset), then set what is needed; a NULL `extras` argument means none.
+ *   seqlens_q, seqlens_k  device int32 [B] per-batch valid query rows / keys
+ *                         (as in attn_fwd_varlen / attn_decode_splitkv_varlen;
+ *                         seqlens_q is for the forward only); NULL = all.
+ *   bias                  device bf16 additive attention bias, laid out
+ *                         [bias_b, bias_h, Sq, Sk] row-major, 2-byte aligned,
+ *                         with bias_b in {1, B} and bias_h in {1, Hq} (1 =
+ *                         broadcast over that dimension).  It is added to the
+ *                         scaled scores before the causal mask:
+ *                         x_ij = scale * q_i.k_j + bias[b', h', i, j], with
+ *                         b' = b unless bias_b == 1 and h' = hq unless
+ *                         bias_h == 1 ("[onnxruntime] WebGPU FlashAttention:
+ *                         kernel fusion and variable sequence length",
+ *                         section 1: the fused decode applies the attention
+ *                         bias with the mask; attn_bias_dim0/dim1 broadcast).
+ *                         LSE is over these x.  A -inf bias entry masks the
+ *                         key.  NULL = no bias.
+ */
+typedef struct {
+  const int* seqlens_q;
+  const int* seqlens_k;
+  const void* bias;
+  int bias_b;
+  int bias_h;
+} attn_extras_t;
+
+/*
  * Prefill / general forward.  Computes o (and lse when non-NULL) for any
  * Sq >= 0, Sk >= 0.  Work items are (b, hq, block of 256 query rows); each
  * visits only the key blocks its causal mask leaves visible ("FlashAttention-2"
@@ -84,6 +112,17 @@ enum { ATTN_CAUSAL_NONE = 0, ATTN_CAUSAL_TOP_LEFT = 1, ATTN_CAUSAL_BOTTOM_RIGHT 
  */
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                        int Sq, int Sk, int d, float scale, int causal, void* stream);
+
+/*
+ * attn_fwd with the optional inputs of attn_extras_t (per-batch lengths as in
+ * attn_fwd_varlen, additive bias; `extras` may be NULL).  With a bias the
+ * forward also needs Sk % 8 == 0 and a 16-byte aligned bias (it reads bias
+ * rows in 16-byte pieces), else ATTN_ERR_ALIGN; invalid bias dims give
+ * ATTN_ERR_SHAPE.
+ */
+attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                          int Sq, int Sk, int d, float scale, int causal, const attn_extras_t* extras,
+                          void* stream);
 
 /*
  * Forward over a batch of sequences of different lengths, held padded:
@@ -172,6 +211,16 @@ attn_status_t attn_decode_splitkv_varlen(const void* q, const void* k_cache, con
                                          const int* seqlens_k, void* o, float* lse, int B, int Hq, int Hkv, int Sq,
                                          int Sk_capacity, int d, float scale, int causal, int num_splits,
                                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_decode_splitkv with the optional inputs of attn_extras_t (per-batch
+ * key lengths, additive bias; `extras` may be NULL).  An invalid extras field
+ * returns ATTN_ERR_SHAPE (bias dims, or seqlens_q given) or ATTN_ERR_ALIGN.
+ */
+attn_status_t attn_decode_splitkv_ex(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                                     int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale, int causal,
+                                     int num_splits, void* workspace, size_t workspace_bytes,
+                                     const attn_extras_t* extras, void* stream);
 
 /*
  * Split-KV decode that allocates nothing and takes no workspace -- for callers

@@ -19,9 +19,16 @@ STATUS_NAMES = {
     13: "ATTN_ERR_SEQLEN",
 }
 STATIC_SCRATCH_BYTES = 16 << 20
-EXPORTS = ("attn_fwd", "attn_fwd_varlen", "attn_decode_num_splits", "attn_decode_workspace_size", "attn_decode_splitkv",
-           "attn_decode_splitkv_varlen", "attn_decode_splitkv_static", "attn_status_string",
+EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_fwd_varlen", "attn_decode_num_splits", "attn_decode_workspace_size", "attn_decode_splitkv",
+           "attn_decode_splitkv_varlen", "attn_decode_splitkv_ex", "attn_decode_splitkv_static",
+           "attn_status_string",
            "attn_check_device_error", "attn_version")
+
+class Extras(ctypes.Structure):
+    """attn_extras_t of the C ABI."""
+    _fields_ = [("seqlens_q", ctypes.c_void_p), ("seqlens_k", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+                ("bias_b", ctypes.c_int), ("bias_h", ctypes.c_int)]
+
 
 _lock = threading.Lock()
 _lib = None
@@ -42,6 +49,11 @@ def _declare(lib):
     P, I, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.attn_fwd.restype = I
+    EP = ctypes.POINTER(Extras)
+    lib.attn_fwd_ex.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, EP, P]
+    lib.attn_fwd_ex.restype = I
+    lib.attn_decode_splitkv_ex.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, P, SZ, EP, P]
+    lib.attn_decode_splitkv_ex.restype = I
     lib.attn_fwd_varlen.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.attn_fwd_varlen.restype = I
     lib.attn_decode_num_splits.argtypes = [I, I, I, I, I, I]

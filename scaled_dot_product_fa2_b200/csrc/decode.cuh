@@ -31,6 +31,9 @@ struct DecodeParams {
   CUtensorMap tm_v;       // [B*Hkv][Sk][d]
   const uint16_t* q;      // [B, Hq, Sq, d] bf16 bits
   const int* seqlens_k;   // [B] valid keys of each batch's cache (device), or nullptr: all Sk
+  const uint16_t* bias;   // bf16 additive bias [bias_b][bias_h][Sq][Sk], or nullptr
+  int64_t bias_sb, bias_sh;  // its batch and head strides in elements (0 where it broadcasts)
+  float inv_scale;        // 1 / scale: the bias enters the raw scores as bias / scale
   float* part_o;          // [B*Hq*Sq][nsplit][d]  locally normalised partial outputs
   float2* part_ml;        // [B*Hq*Sq][nsplit]     (local max of scale*q.k, local sum)
   int B, Hq, Hkv, Sq, Sk, group;
@@ -185,13 +188,19 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
       qf[ks][3] = v_hi ? q_hi[(ks * 16 + 8 + qc) >> 1] : 0u;
     }
   }
-  // causal limit per fragment row: the last key each row may see
+  // causal limit per fragment row: the last key each row may see; and the
+  // row of the bias (if any) that belongs to it
   int lim[2];
+  const uint16_t* brow[2] = {nullptr, nullptr};
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int lr = rg * kDecRows + qr + 8 * h;  // local row = g*Sq + i
     const int i = lr % p.Sq;
     lim[h] = p.causal ? min(L - 1, i + coff) : L - 1;
+    if (p.bias != nullptr && lr < rows_total) {
+      const int hq = hkv * p.group + lr / p.Sq;
+      brow[h] = p.bias + b * p.bias_sb + hq * p.bias_sh + static_cast<int64_t>(i) * p.Sk;
+    }
   }
 
   float o[D / 8][4];
@@ -223,8 +232,20 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
         mma_bf16_16816(sc[1], qf[ks], b2, b3);
       }
     }
-    // ---- mask, online softmax (rows qr and qr+8 of this thread)
+    // ---- bias, mask, online softmax (rows qr and qr+8 of this thread)
     const int key0 = (tile_begin + it) * kDecKeys + kb;
+    if (p.bias != nullptr) {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int key = key0 + nt * 8 + qc;  // this thread's keys key, key + 1
+          if (brow[h] != nullptr) {
+            if (key < p.Sk) sc[nt][2 * h] += bf16_bits_to_float(__ldg(brow[h] + key)) * p.inv_scale;
+            if (key + 1 < p.Sk) sc[nt][2 * h + 1] += bf16_bits_to_float(__ldg(brow[h] + key + 1)) * p.inv_scale;
+          }
+        }
+    }
     if (key0 + 15 > min(lim[0], lim[1])) {
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)

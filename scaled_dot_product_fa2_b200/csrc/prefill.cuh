@@ -65,6 +65,9 @@ struct PrefillParams {
   float* lse;        // [B*Hq*Sq] or nullptr
   const int* seqlens_q;  // [B] valid query rows of each batch (device), or nullptr: all Sq
   const int* seqlens_k;  // [B] valid keys of each batch (device), or nullptr: all Sk
+  const uint16_t* bias;  // bf16 additive bias [bias_b][bias_h][Sq][Sk] (Sk % 8 == 0), or nullptr
+  int64_t bias_sb, bias_sh;  // its batch and head strides in elements (0 where it broadcasts)
+  float inv_scale;       // 1 / scale: the bias enters the raw scores as bias / scale
   int B, Hq, Hkv, Sq, Sk;
   int group;          // Hq / Hkv
   int causal;         // 0 none, 1 top-left, 2 bottom-right
@@ -87,6 +90,11 @@ constexpr int kLaunchRegs = 168;  // 3 warps per SM sub-partition: 3*32*168 <= 1
 constexpr int kSoftmaxRegs = 216;
 constexpr int kCtrlRegs = 72;
 static_assert(256 * kSoftmaxRegs + 128 * kCtrlRegs == kPrefillThreads * kLaunchRegs,
+              "register split must equal the launch allocation");
+// The bias variant's softmax holds a tile of bias besides the scores.
+constexpr int kSoftmaxRegsBias = 224;
+constexpr int kCtrlRegsBias = 56;
+static_assert(256 * kSoftmaxRegsBias + 128 * kCtrlRegsBias == kPrefillThreads * kLaunchRegs,
               "register split must equal the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest P kept unrescaled
 
@@ -193,7 +201,25 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint6
   }
 }
 
-template <int D, int NS>
+// Bias of one query row for keys k0 + 8*c .. k0 + 8*c + 7, c in [C0, C0 + 8),
+// as bf16 pairs (row or keys out of the bias give zeros: those scores are
+// masked or never written).  The row's address is recomputed at each call: a
+// pointer kept live across the softmax step would cost registers it needs.
+template <int C0>
+__device__ __forceinline__ void load_bias_chunks(const PrefillParams& p, int bh, int row, int k0, uint4 (&bz)[16]) {
+  const int b = bh / p.Hq;
+  const uint16_t* brow = p.bias + b * p.bias_sb + (bh - b * p.Hq) * p.bias_sh + static_cast<int64_t>(row) * p.Sk;
+#pragma unroll
+  for (int c8 = C0; c8 < C0 + 8; ++c8) {
+    const int key = k0 + c8 * 8;
+    bz[c8] = (row < p.Sq && key < p.Sk) ? __ldg(reinterpret_cast<const uint4*>(brow + key))
+                                         : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// BIAS: add the additive attention bias to the scores (a separate
+// instantiation, so the common path carries none of its loads).
+template <int D, int NS, bool BIAS>
 __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
   using Cfg = PrefillCfg<D, NS>;
   extern __shared__ uint8_t smem_raw[];
@@ -248,7 +274,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
   const uint32_t tmem = *tmem_slot;
   if (warp >= 8) {
     // Warpgroup 2 (control): every warp runs the same setmaxnreg first.
-    regs_decrease<kCtrlRegs>();
+    regs_decrease<BIAS ? kCtrlRegsBias : kCtrlRegs>();
     if (warp == kLoadWarp) {
       // ------------------------------------------------------ TMA producer
       // Per unit: K_0, V_0 through the ring, then Q_0, Q_1 (each once the
@@ -412,7 +438,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
     }
   } else {
     // Warpgroups 0 and 1: softmax / epilogue for query tile 0 and 1.
-    regs_increase<kSoftmaxRegs>();
+    regs_increase<BIAS ? kSoftmaxRegsBias : kSoftmaxRegs>();
     const int t = warp >> 2;      // query tile 0 or 1
     const int wq = warp & 3;      // TMEM lane quarter of this warp
     const int r_in_tile = wq * 32 + lane;
@@ -437,16 +463,46 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
 
 #pragma unroll 1
       for (int j = 0; j < n; ++j, ++sj) {
+        // The bias of this key tile's first 64 keys is fetched before the wait
+        // for S, so its latency overlaps the wait; the second 64 right after
+        // (keys past Sk read nothing: they are masked).
+        uint4 bz[BIAS ? 16 : 1];
+        if constexpr (BIAS) load_bias_chunks<0>(p, u.bh, row, j * kBlockN, bz);
         if (!mbar_wait(s_full(t), sj & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         uint32_t sv[128];
+        if constexpr (!BIAS) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[q * 32]));
-        tmem_wait_ld();
-
+          for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[q * 32]));
+          tmem_wait_ld();
+        } else {
+          // S in two 64-column halves, each given its bias as soon as it lands
+          // (fewer registers live at once than all of S plus all of the bias).
+          const float2 is2 = make_float2(p.inv_scale, p.inv_scale);
+          load_bias_chunks<8>(p, u.bh, row, j * kBlockN, bz);
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            tmem_ld32(tS + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[half * 64]));
+            tmem_ld32(tS + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[half * 64 + 32]));
+            tmem_wait_ld();
+#pragma unroll
+            for (int c8 = half * 8; c8 < half * 8 + 8; ++c8) {
+              const uint32_t w[4] = {bz[c8].x, bz[c8].y, bz[c8].z, bz[c8].w};
+#pragma unroll
+              for (int u2 = 0; u2 < 4; ++u2) {
+                const int e = c8 * 8 + u2 * 2;
+                const float2 bb = make_float2(__uint_as_float(w[u2] << 16), __uint_as_float(w[u2] & 0xFFFF0000u));
+                const float2 r =
+                    __ffma2_rn(bb, is2, make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])));
+                sv[e] = __float_as_uint(r.x);
+                sv[e + 1] = __float_as_uint(r.y);
+              }
+            }
+          }
+        }
         const int k0 = j * kBlockN;
         const bool need_mask = (k0 + kBlockN > u.Lk) || (p.causal && k0 + kBlockN - 1 > row0 + u.coff);
         if (need_mask) {

@@ -45,6 +45,26 @@ attn_status_t check_common(const void* q, const void* k, const void* v, const vo
   return ATTN_OK;
 }
 
+// The optional inputs of the *_ex entry points (nullptr: none of them).
+attn_status_t check_extras(const attn_extras_t* ex, int B, int Hq, bool allow_seqlens_q) {
+  if (ex == nullptr) return ATTN_OK;
+  if (ex->seqlens_q != nullptr && (!allow_seqlens_q || !aligned(ex->seqlens_q, 4)))
+    return allow_seqlens_q ? ATTN_ERR_ALIGN : ATTN_ERR_SHAPE;
+  if (ex->seqlens_k != nullptr && !aligned(ex->seqlens_k, 4)) return ATTN_ERR_ALIGN;
+  if (ex->bias != nullptr) {
+    if (!(ex->bias_b == 1 || ex->bias_b == B) || !(ex->bias_h == 1 || ex->bias_h == Hq)) return ATTN_ERR_SHAPE;
+    if (!aligned(ex->bias, 2)) return ATTN_ERR_ALIGN;
+  }
+  return ATTN_OK;
+}
+
+// Element strides of a bias [bias_b, bias_h, Sq, Sk]: 0 along a broadcast dim.
+void bias_strides(const attn_extras_t* ex, int Sq, int Sk, int64_t* sb, int64_t* sh) {
+  const int64_t plane = static_cast<int64_t>(Sq) * Sk;
+  *sh = (ex->bias_h == 1) ? 0 : plane;
+  *sb = (ex->bias_b == 1) ? 0 : plane * ex->bias_h;
+}
+
 float effective_scale(float scale, int d) { return scale == 0.f ? 1.f / std::sqrt(static_cast<float>(d)) : scale; }
 
 int causal_offset(int causal, int Sq, int Sk) { return causal == ATTN_CAUSAL_BOTTOM_RIGHT ? Sk - Sq : 0; }
@@ -154,7 +174,7 @@ attn_status_t launch_fill_empty(void* o, float* lse, int64_t rows, int d, cudaSt
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D, int NS>
+template <int D, int NS, bool BIAS>
 attn_status_t launch_prefill(const PrefillParams& prm, int grid, int dev, cudaStream_t st) {
   static bool smem_done[kMaxDevices] = {};
   static std::mutex mu;
@@ -166,17 +186,17 @@ attn_status_t launch_prefill(const PrefillParams& prm, int grid, int dev, cudaSt
       // kLaunchRegs per thread; launching with any other allocation could make
       // setmaxnreg.inc wait forever, so refuse instead.
       cudaFuncAttributes fa;
-      if (cudaFuncGetAttributes(&fa, prefill_kernel<D, NS>) != cudaSuccess || fa.numRegs != kLaunchRegs)
+      if (cudaFuncGetAttributes(&fa, prefill_kernel<D, NS, BIAS>) != cudaSuccess || fa.numRegs != kLaunchRegs)
         return ATTN_ERR_CUDA;
     }
-    if (!set_smem(prefill_kernel<D, NS>, Cfg::kSmemBytes, dev, smem_done)) return ATTN_ERR_CUDA;
+    if (!set_smem(prefill_kernel<D, NS, BIAS>, Cfg::kSmemBytes, dev, smem_done)) return ATTN_ERR_CUDA;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kPrefillThreads);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = st;
-  return cudaLaunchKernelEx(&cfg, prefill_kernel<D, NS>, prm) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return cudaLaunchKernelEx(&cfg, prefill_kernel<D, NS, BIAS>, prm) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 // ------------------------------------------------------------ decode split policy
@@ -284,11 +304,15 @@ using namespace sdpa;
 
 extern "C" {
 
-static attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int* seqlens_q,
-                              const int* seqlens_k, void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Sk,
-                              int d, float scale, int causal, void* stream) {
+static attn_status_t fwd_impl(const void* q, const void* k, const void* v, const attn_extras_t* ex, void* o,
+                              float* lse, int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale, int causal,
+                              void* stream) {
   attn_status_t s = check_common(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
   if (s != ATTN_OK) return s;
+  if ((s = check_extras(ex, B, Hq, true)) != ATTN_OK) return s;
+  const bool has_bias = ex != nullptr && ex->bias != nullptr;
+  // the forward reads bias rows with 16-byte loads: rows must be 16-byte aligned
+  if (has_bias && (Sk % 8 != 0 || !aligned(ex->bias, 16))) return ATTN_ERR_ALIGN;
   if (B == 0 || Sq == 0) return ATTN_OK;
   int dev = 0, sms = 0;
   if ((s = current_device(&dev, &sms)) != ATTN_OK) return s;
@@ -305,8 +329,12 @@ static attn_status_t fwd_impl(const void* q, const void* k, const void* v, const
     return ATTN_ERR_CUDA;
   prm.o = static_cast<uint16_t*>(o);
   prm.lse = lse;
-  prm.seqlens_q = seqlens_q;
-  prm.seqlens_k = seqlens_k;
+  prm.seqlens_q = ex ? ex->seqlens_q : nullptr;
+  prm.seqlens_k = ex ? ex->seqlens_k : nullptr;
+  if (has_bias) {
+    prm.bias = static_cast<const uint16_t*>(ex->bias);
+    bias_strides(ex, Sq, Sk, &prm.bias_sb, &prm.bias_sh);
+  }
   prm.B = B;
   prm.Hq = Hq;
   prm.Hkv = Hkv;
@@ -319,18 +347,29 @@ static attn_status_t fwd_impl(const void* q, const void* k, const void* v, const
   prm.lpt = causal != ATTN_CAUSAL_NONE ? 1 : 0;
   prm.scale = sc;
   prm.scale_log2 = sc * 1.4426950408889634f;
+  prm.inv_scale = 1.f / sc;
   const int64_t units = static_cast<int64_t>(B) * Hq * prm.num_units;
   if (units > INT_MAX / 2) return ATTN_ERR_SHAPE;
   prm.total_units = static_cast<int>(units);
   // Persistent grid: one CTA per SM (the kernel's shared memory allows one).
   const int64_t grid = std::min<int64_t>(units, sms);
-  if (d == 128) return launch_prefill<128, kStagesD128>(prm, static_cast<int>(grid), dev, st);
-  return launch_prefill<64, kStagesD64>(prm, static_cast<int>(grid), dev, st);
+  if (d == 128) {
+    return has_bias ? launch_prefill<128, kStagesD128, true>(prm, static_cast<int>(grid), dev, st)
+                    : launch_prefill<128, kStagesD128, false>(prm, static_cast<int>(grid), dev, st);
+  }
+  return has_bias ? launch_prefill<64, kStagesD64, true>(prm, static_cast<int>(grid), dev, st)
+                  : launch_prefill<64, kStagesD64, false>(prm, static_cast<int>(grid), dev, st);
 }
 
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                        int Sq, int Sk, int d, float scale, int causal, void* stream) {
-  return fwd_impl(q, k, v, nullptr, nullptr, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal, stream);
+  return fwd_impl(q, k, v, nullptr, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal, stream);
+}
+
+attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                          int Sq, int Sk, int d, float scale, int causal, const attn_extras_t* extras,
+                          void* stream) {
+  return fwd_impl(q, k, v, extras, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal, stream);
 }
 
 attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, const int* seqlens_q,
@@ -340,7 +379,11 @@ attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, const
     if (seqlens_q == nullptr || seqlens_k == nullptr) return ATTN_ERR_NULL;
     if (!aligned(seqlens_q, 4) || !aligned(seqlens_k, 4)) return ATTN_ERR_ALIGN;
   }
-  return fwd_impl(q, k, v, seqlens_q, seqlens_k, o, lse, B, Hq, Hkv, Sq_max, Sk_max, d, scale, causal, stream);
+  attn_extras_t ex;
+  std::memset(&ex, 0, sizeof(ex));
+  ex.seqlens_q = seqlens_q;
+  ex.seqlens_k = seqlens_k;
+  return fwd_impl(q, k, v, &ex, o, lse, B, Hq, Hkv, Sq_max, Sk_max, d, scale, causal, stream);
 }
 
 int attn_decode_num_splits(int B, int Hq, int Hkv, int Sq, int Sk, int d) {
@@ -356,11 +399,13 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int d,
   return decode_ws_bytes(B, Hq, Sq, d, ns);
 }
 
-static attn_status_t decode_impl(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k,
+static attn_status_t decode_impl(const void* q, const void* k_cache, const void* v_cache, const attn_extras_t* ex,
                                  void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale,
                                  int causal, int num_splits, void* workspace, size_t workspace_bytes, void* stream) {
   attn_status_t s = check_common(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
   if (s != ATTN_OK) return s;
+  if ((s = check_extras(ex, B, Hq, false)) != ATTN_OK) return s;
+  const int* seqlens_k = ex ? ex->seqlens_k : nullptr;
   if (num_splits < 0) return ATTN_ERR_SHAPE;
   if (B == 0 || Sq == 0) return ATTN_OK;
   int dev = 0, sms = 0;
@@ -388,6 +433,10 @@ static attn_status_t decode_impl(const void* q, const void* k_cache, const void*
   float2* part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + rows * ns * d * sizeof(float));
   prm.q = static_cast<const uint16_t*>(q);
   prm.seqlens_k = seqlens_k;
+  if (ex != nullptr && ex->bias != nullptr) {
+    prm.bias = static_cast<const uint16_t*>(ex->bias);
+    bias_strides(ex, Sq, Sk, &prm.bias_sb, &prm.bias_sh);
+  }
   prm.part_o = part_o;
   prm.part_ml = part_ml;
   prm.B = B;
@@ -403,6 +452,7 @@ static attn_status_t decode_impl(const void* q, const void* k_cache, const void*
   prm.row_groups = rg;
   prm.scale = sc;
   prm.scale_log2 = sc * 1.4426950408889634f;
+  prm.inv_scale = 1.f / sc;
   const int64_t grid = static_cast<int64_t>(B) * Hkv * ns * rg;
   if (grid > INT_MAX || (rows + 3) / 4 > INT_MAX) return ATTN_ERR_SHAPE;
   if (d == 128) return launch_decode<128>(prm, static_cast<int>(grid), part_o, part_ml, o, lse, rows, dev, st);
@@ -424,8 +474,19 @@ attn_status_t attn_decode_splitkv_varlen(const void* q, const void* k_cache, con
     if (seqlens_k == nullptr) return ATTN_ERR_NULL;
     if (!aligned(seqlens_k, 4)) return ATTN_ERR_ALIGN;
   }
-  return decode_impl(q, k_cache, v_cache, seqlens_k, o, lse, B, Hq, Hkv, Sq, Sk_capacity, d, scale, causal,
-                     num_splits, workspace, workspace_bytes, stream);
+  attn_extras_t ex;
+  std::memset(&ex, 0, sizeof(ex));
+  ex.seqlens_k = seqlens_k;
+  return decode_impl(q, k_cache, v_cache, &ex, o, lse, B, Hq, Hkv, Sq, Sk_capacity, d, scale, causal, num_splits,
+                     workspace, workspace_bytes, stream);
+}
+
+attn_status_t attn_decode_splitkv_ex(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                                     int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale, int causal,
+                                     int num_splits, void* workspace, size_t workspace_bytes,
+                                     const attn_extras_t* extras, void* stream) {
+  return decode_impl(q, k_cache, v_cache, extras, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal, num_splits,
+                     workspace, workspace_bytes, stream);
 }
 
 const char* attn_status_string(attn_status_t status) {

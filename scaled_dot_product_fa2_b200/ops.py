@@ -6,6 +6,8 @@ pointers plus the current CUDA stream.
 """
 from __future__ import annotations
 
+import ctypes
+
 import torch
 
 from . import _lib
@@ -60,21 +62,41 @@ def _outputs(q, out, lse, want_lse):
     return out, lse
 
 
+def _bias_extras(bias, B, Hq, Sq, Sk, device, ex=None):
+    """attn_extras_t carrying a bf16 bias [1|B, 1|Hq, Sq, Sk] (or None)."""
+    ex = ex if ex is not None else _lib.Extras()
+    if bias is None:
+        return ex
+    _check_tensor("bias", bias, torch.bfloat16, 4)
+    if (bias.shape[0] not in (1, B) or bias.shape[1] not in (1, Hq) or tuple(bias.shape[2:]) != (Sq, Sk)
+            or bias.device != device):
+        raise ValueError(f"bias must be [1|B, 1|Hq, Sq, Sk] on q's device, got {tuple(bias.shape)}")
+    ex.bias = bias.data_ptr()
+    ex.bias_b = int(bias.shape[0])
+    ex.bias_h = int(bias.shape[1])
+    return ex
+
+
 def attn_fwd(q, k, v, causal: int = CAUSAL_NONE, scale: float = 0.0, out=None, lse=None,
-             return_lse: bool = True):
-    """O = softmax(scale * q k^T + mask) v through ``attn_fwd`` of the C ABI.
+             return_lse: bool = True, bias=None):
+    """O = softmax(scale * q k^T + bias + mask) v through the C ABI.
 
     q [B,Hq,Sq,d], k/v [B,Hkv,Sk,d] bf16 contiguous CUDA tensors; ``scale=0``
-    means 1/sqrt(d).  Returns (o, lse) with lse fp32 [B,Hq,Sq] (None when
+    means 1/sqrt(d); ``bias`` an optional bf16 [1|B, 1|Hq, Sq, Sk] tensor
+    (``attn_fwd_ex``).  Returns (o, lse) with lse fp32 [B,Hq,Sq] (None when
     ``return_lse`` is False and no ``lse`` buffer was given).
     """
     B, Hq, Hkv, Sq, Sk, d = _shapes(q, k, v)
     out, lse = _outputs(q, out, lse, return_lse)
     lib = _lib.get()
     with torch.cuda.device(q.device):
-        st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                          lse.data_ptr() if lse is not None else None,
-                          B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal), _stream_handle(q.device))
+        args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr() if lse is not None else None,
+                B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal))
+        if bias is None:
+            st = lib.attn_fwd(*args, _stream_handle(q.device))
+        else:
+            ex = _bias_extras(bias, B, Hq, Sq, Sk, q.device)
+            st = lib.attn_fwd_ex(*args, ctypes.byref(ex), _stream_handle(q.device))
     _lib.check(st, "attn_fwd")
     return out, lse
 
@@ -127,8 +149,14 @@ def decode_workspace(q, k_cache, num_splits: int = 0) -> torch.Tensor:
 
 
 def attn_decode_splitkv(q, k_cache, v_cache, causal: int = CAUSAL_BOTTOM_RIGHT, scale: float = 0.0,
-                        num_splits: int = 0, workspace=None, out=None, lse=None, return_lse: bool = True):
-    """Split-KV decode through ``attn_decode_splitkv`` of the C ABI.  Returns (o, lse)."""
+                        num_splits: int = 0, workspace=None, out=None, lse=None, return_lse: bool = True,
+                        bias=None, seqlens_k=None):
+    """Split-KV decode through the C ABI (``attn_decode_splitkv``, or
+    ``attn_decode_splitkv_ex`` when a bf16 ``bias`` [1|B, 1|Hq, Sq, Sk] or
+    int32 ``seqlens_k`` [B] is given).  Returns (o, lse)."""
+    if bias is not None or seqlens_k is not None:
+        return _decode_ex(q, k_cache, v_cache, causal, scale, num_splits, workspace, out, lse, return_lse, bias,
+                          seqlens_k)
     B, Hq, Hkv, Sq, Sk, d = _shapes(q, k_cache, v_cache)
     out, lse = _outputs(q, out, lse, return_lse)
     if workspace is None:
@@ -143,6 +171,28 @@ def attn_decode_splitkv(q, k_cache, v_cache, causal: int = CAUSAL_BOTTOM_RIGHT, 
                                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                      _stream_handle(q.device))
     _lib.check(st, "attn_decode_splitkv")
+    return out, lse
+
+
+def _decode_ex(q, k_cache, v_cache, causal, scale, num_splits, workspace, out, lse, return_lse, bias, seqlens_k):
+    B, Hq, Hkv, Sq, Sk, d = _shapes(q, k_cache, v_cache)
+    ex = _bias_extras(bias, B, Hq, Sq, Sk, q.device)
+    if seqlens_k is not None:
+        _check_lengths("seqlens_k", seqlens_k, B, q.device)
+        ex.seqlens_k = seqlens_k.data_ptr()
+    out, lse = _outputs(q, out, lse, return_lse)
+    if workspace is None:
+        workspace = decode_workspace(q, k_cache, num_splits)
+    if workspace.device != q.device or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous buffer on q's device")
+    lib = _lib.get()
+    with torch.cuda.device(q.device):
+        st = lib.attn_decode_splitkv_ex(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
+                                        lse.data_ptr() if lse is not None else None,
+                                        B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal), int(num_splits),
+                                        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                        ctypes.byref(ex), _stream_handle(q.device))
+    _lib.check(st, "attn_decode_splitkv_ex")
     return out, lse
 
 

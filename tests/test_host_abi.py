@@ -124,6 +124,29 @@ def test_varlen_forward_rejects_bad_lengths_pointers_on_host(lib):
     assert lib.attn_fwd_varlen(None, None, None, None, None, None, None, 0, 4, 2, 64, 64, 128, 0.0, 0, None) == 0
 
 
+def test_extras_are_validated_on_host(lib):
+    from scaled_dot_product_fa2_b200._lib import Extras
+    ex = Extras()
+    ex.bias = P
+    ex.bias_b, ex.bias_h = 1, 1
+    fwd = lambda Sk, e: lib.attn_fwd_ex(P, P, P, P, None, 2, 4, 2, 64, Sk, 128, 0.0, 0, ctypes.byref(e), None)
+    assert fwd(12, ex) == 5          # forward bias rows must be 16-byte aligned: Sk % 8 == 0
+    ex.bias_b = 3
+    assert fwd(64, ex) == 2          # bias_b must be 1 or B
+    ex.bias_b, ex.bias_h = 2, 2
+    assert fwd(64, ex) == 2          # bias_h must be 1 or Hq
+    ex.bias_h = 4
+    ex.bias = P + 2
+    assert fwd(64, ex) == 5          # 16-byte aligned bias base for the forward
+    dec = lambda e: lib.attn_decode_splitkv_ex(P, P, P, P, None, 2, 4, 2, 1, 256, 128, 0.0, 2, 0, P,
+                                               1 << 30, ctypes.byref(e), None)
+    ex.bias = P + 1
+    assert dec(ex) == 5              # 2-byte alignment for the decode's bias
+    ex2 = Extras()
+    ex2.seqlens_q = P
+    assert dec(ex2) == 2             # the decode takes no query lengths
+
+
 def test_ptxas_report_checker():
     regs = build.PREFILL_LAUNCH_REGS
     ok = ("ptxas info    : Compiling entry function '_ZN4sdpa14prefill_kernelILi128ELi4EEEvNS_13PrefillParamsE'\n"
@@ -134,6 +157,12 @@ def test_ptxas_report_checker():
         build.check_ptxas_report(ok.replace(f"Used {regs}", f"Used {regs - 8}"))
     with pytest.raises(RuntimeError):
         build.check_ptxas_report(ok.replace("0 bytes spill stores", "8 bytes spill stores"))
+    # the bias instantiation may spill a few bytes, nothing more
+    bias = ok.replace("Li4EEEv", "Li4ELb1EEEv")
+    build.check_ptxas_report(bias.replace("0 bytes spill stores, 0 bytes spill loads",
+                                          "4 bytes spill stores, 16 bytes spill loads"))
+    with pytest.raises(RuntimeError):
+        build.check_ptxas_report(bias.replace("0 bytes spill stores", "64 bytes spill stores"))
 
 
 def test_decode_split_policy_fills_one_wave(lib):
