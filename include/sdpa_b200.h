@@ -77,6 +77,14 @@ typedef enum {
 enum { ATTN_CAUSAL_NONE = 0, ATTN_CAUSAL_TOP_LEFT = 1, ATTN_CAUSAL_BOTTOM_RIGHT = 2 };
 
 /*
+ * Tensor layouts (attn_extras_t.layout): BHSD is [B, H, S, d] (heads outer,
+ * the default everywhere); BSHD is [B, S, H, d] (tokens outer: the
+ * non-"BNSH" Q format of the onnxruntime WebGPU decode page, section 2).
+ * Both contiguous with d innermost.
+ */
+enum { ATTN_LAYOUT_BHSD = 0, ATTN_LAYOUT_BSHD = 1 };
+
+/*
  * Optional inputs of attn_fwd_ex and attn_decode_splitkv_ex.  Zero-initialise
  * (memset), then set what is needed; a NULL `extras` argument means none.
  *   seqlens_q, seqlens_k  device int32 [B] per-batch valid query rows / keys
@@ -95,6 +103,10 @@ enum { ATTN_CAUSAL_NONE = 0, ATTN_CAUSAL_TOP_LEFT = 1, ATTN_CAUSAL_BOTTOM_RIGHT 
  *                         bias with the mask; attn_bias_dim0/dim1 broadcast).
  *                         LSE is over these x.  A -inf bias entry masks the
  *                         key.  NULL = no bias.
+ *   layout                ATTN_LAYOUT_BHSD (0) or ATTN_LAYOUT_BSHD: the layout
+ *                         of q, k, v and o for the forward, of q and o for the
+ *                         decode (its K/V cache is always [B, Hkv, S, d]).  lse,
+ *                         the lengths and the bias keep their layouts.
  */
 typedef struct {
   const int* seqlens_q;
@@ -102,6 +114,7 @@ typedef struct {
   const void* bias;
   int bias_b;
   int bias_h;
+  int layout;
 } attn_extras_t;
 
 /*

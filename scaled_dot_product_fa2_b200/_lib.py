@@ -27,7 +27,7 @@ EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_fwd_varlen", "attn_decode_num_splits
 class Extras(ctypes.Structure):
     """attn_extras_t of the C ABI."""
     _fields_ = [("seqlens_q", ctypes.c_void_p), ("seqlens_k", ctypes.c_void_p), ("bias", ctypes.c_void_p),
-                ("bias_b", ctypes.c_int), ("bias_h", ctypes.c_int)]
+                ("bias_b", ctypes.c_int), ("bias_h", ctypes.c_int), ("layout", ctypes.c_int)]
 
 
 _lock = threading.Lock()

@@ -29,7 +29,8 @@ namespace sdpa {
 struct DecodeParams {
   CUtensorMap tm_k;       // [B*Hkv][Sk][d] bf16, box {64, 64, 1}, 128-byte swizzle
   CUtensorMap tm_v;       // [B*Hkv][Sk][d]
-  const uint16_t* q;      // [B, Hq, Sq, d] bf16 bits
+  const uint16_t* q;      // bf16 bits; element (b, h, i, c) at b*q_sb + h*q_sh + i*q_sr + c
+  int64_t q_sb, q_sh, q_sr;
   const int* seqlens_k;   // [B] valid keys of each batch's cache (device), or nullptr: all Sk
   const uint16_t* bias;   // bf16 additive bias [bias_b][bias_h][Sq][Sk], or nullptr
   int64_t bias_sb, bias_sh;  // its batch and head strides in elements (0 where it broadcasts)
@@ -177,9 +178,15 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
   {
     const int r_lo = rg * kDecRows + qr;
     const int r_hi = r_lo + 8;
-    const uint32_t* q_lo = reinterpret_cast<const uint32_t*>(p.q + (row_base + r_lo) * D);
-    const uint32_t* q_hi = reinterpret_cast<const uint32_t*>(p.q + (row_base + r_hi) * D);
     const bool v_lo = r_lo < rows_total, v_hi = r_hi < rows_total;
+    // local row g*Sq + i of this KV head -> query head hkv*group + g, row i
+    auto q_row = [&](int lr) {
+      const int g = lr / p.Sq;
+      return reinterpret_cast<const uint32_t*>(p.q + b * p.q_sb + (hkv * p.group + g) * p.q_sh +
+                                               (lr - g * p.Sq) * p.q_sr);
+    };
+    const uint32_t* q_lo = q_row(v_lo ? r_lo : 0);
+    const uint32_t* q_hi = q_row(v_hi ? r_hi : 0);
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
       qf[ks][0] = v_lo ? q_lo[(ks * 16 + qc) >> 1] : 0u;
@@ -383,11 +390,17 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
 // The kernel is launched as a programmatic dependent of the split kernel: it
 // may start while the split kernel's last CTAs run, and waits for that
 // grid's completion (and the visibility of its writes) before reading.
+// Where output row (b*Hq + h)*Sq + i lives: b*sb + h*sh + i*sr elements.
+struct RowLayout {
+  int Hq, Sq;
+  int64_t sb, sh, sr;
+};
+
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ part_o,
                                                              const float2* __restrict__ part_ml,
                                                              uint16_t* __restrict__ out, float* __restrict__ lse,
-                                                             int64_t rows, int nsplit) {
+                                                             int64_t rows, int nsplit, RowLayout ol) {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   constexpr int kPer = D / 32;  // floats per lane: 4 (one 16-byte load) or 2
   constexpr int kUnroll = 8;
@@ -451,7 +464,9 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
     for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
   }
   const float inv = (W > 0.f) ? 1.f / W : 0.f;
-  uint16_t* dst = out + row * D + lane * kPer;
+  const int64_t bh = row / ol.Sq;
+  const int64_t bb = bh / ol.Hq;
+  uint16_t* dst = out + bb * ol.sb + (bh - bb * ol.Hq) * ol.sh + (row - bh * ol.Sq) * ol.sr + lane * kPer;
   if constexpr (kPer == 4) {
     *reinterpret_cast<uint2*>(dst) =
         make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));

@@ -58,10 +58,13 @@
 namespace sdpa {
 
 struct PrefillParams {
-  CUtensorMap tm_q;  // [B*Hq][Sq][d] bf16, box {64, 128, 1}, 128-byte swizzle
-  CUtensorMap tm_k;  // [B*Hkv][Sk][d]
-  CUtensorMap tm_v;  // [B*Hkv][Sk][d]
-  uint16_t* o;       // [B*Hq][Sq][d] bf16 bits
+  // 4-D maps (d, S, H, B) over q, k, v whatever their layout (the strides
+  // carry it); box {64, 128, 1, 1}, 128-byte swizzle.
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  uint16_t* o;       // bf16 bits; element (b, h, i, c) at b*o_sb + h*o_sh + i*o_sr + c
+  int64_t o_sb, o_sh, o_sr;
   float* lse;        // [B*Hq*Sq] or nullptr
   const int* seqlens_q;  // [B] valid query rows of each batch (device), or nullptr: all Sq
   const int* seqlens_k;  // [B] valid keys of each batch (device), or nullptr: all Sk
@@ -138,7 +141,7 @@ __device__ __forceinline__ void unit_coords(const PrefillParams& p, int idx, int
 }
 
 struct Unit {
-  int bh, bhkv, row0_0, n0, n1, n_max;
+  int bh, b, hq, hkv, row0_0, n0, n1, n_max;
   int Lq, Lk, coff;  // this batch's valid query rows, valid keys, causal offset
 };
 
@@ -153,7 +156,9 @@ __device__ __forceinline__ Unit make_unit(const PrefillParams& p, int idx) {
   unit_coords(p, idx, u.bh, v);
   const int b = u.bh / p.Hq;
   const int hq = u.bh - b * p.Hq;
-  u.bhkv = b * p.Hkv + hq / p.group;
+  u.b = b;
+  u.hq = hq;
+  u.hkv = hq / p.group;
   u.row0_0 = v * 2 * kBlockM;
   u.Lq = batch_length(p.seqlens_q, b, p.Sq);
   u.Lk = batch_length(p.seqlens_k, b, p.Sk);
@@ -296,8 +301,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
             if ((t ? u.n1 : u.n0) > 0) {
               mbar_arrive_expect_tx(q_full(t), Cfg::kTileBytes);
               for (int blk = 0; blk < Cfg::kBlocks; ++blk)
-                tma_load_3d(sQ + t * Cfg::kTileBytes + blk * Cfg::kBlockBytes, &p.tm_q, blk * 64,
-                            u.row0_0 + t * kBlockM, u.bh, q_full(t));
+                tma_load_4d(sQ + t * Cfg::kTileBytes + blk * Cfg::kBlockBytes, &p.tm_q, blk * 64,
+                            u.row0_0 + t * kBlockM, u.hq, u.b, q_full(t));
             } else {
               mbar_arrive(q_full(t));
             }
@@ -331,7 +336,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
             const CUtensorMap* tm = (x & 1) ? &p.tm_v : &p.tm_k;
             const uint32_t dst = sKV + slot * Cfg::kTileBytes;
             for (int blk = 0; blk < Cfg::kBlocks; ++blk)
-              tma_load_3d(dst + blk * Cfg::kBlockBytes, tm, blk * 64, (x >> 1) * kBlockN, u.bhkv, kv_full(slot));
+              tma_load_4d(dst + blk * Cfg::kBlockBytes, tm, blk * 64, (x >> 1) * kBlockN, u.hkv, u.b,
+                          kv_full(slot));
           }
           ++ui;
         }
@@ -588,7 +594,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
         // LSE = -inf.
         const bool empty_row = (m_used == -INFINITY) || !(l > 0.f);
         const float inv_l = empty_row ? 0.f : 1.f / l;
-        uint16_t* dst = p.o + (static_cast<int64_t>(u.bh) * p.Sq + row) * D;
+        uint16_t* dst = p.o + u.b * p.o_sb + u.hq * p.o_sh + row * p.o_sr;
 #pragma unroll 1
         for (int q = 0; q < D / 32; ++q) {
           uint32_t o[32];

@@ -51,6 +51,7 @@ attn_status_t check_extras(const attn_extras_t* ex, int B, int Hq, bool allow_se
   if (ex->seqlens_q != nullptr && (!allow_seqlens_q || !aligned(ex->seqlens_q, 4)))
     return allow_seqlens_q ? ATTN_ERR_ALIGN : ATTN_ERR_SHAPE;
   if (ex->seqlens_k != nullptr && !aligned(ex->seqlens_k, 4)) return ATTN_ERR_ALIGN;
+  if (ex->layout != ATTN_LAYOUT_BHSD && ex->layout != ATTN_LAYOUT_BSHD) return ATTN_ERR_SHAPE;
   if (ex->bias != nullptr) {
     if (!(ex->bias_b == 1 || ex->bias_b == B) || !(ex->bias_h == 1 || ex->bias_h == Hq)) return ATTN_ERR_SHAPE;
     if (!aligned(ex->bias, 2)) return ATTN_ERR_ALIGN;
@@ -139,6 +140,32 @@ bool make_map(CUtensorMap* map, const void* base, int d, int rows, int64_t outer
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Element strides (batch, head, row) of a [B, H, S, d] tensor in `layout`.
+struct Strides {
+  int64_t b, h, r;
+};
+Strides layout_strides(int layout, int H, int S, int d) {
+  if (layout == ATTN_LAYOUT_BSHD) return {static_cast<int64_t>(S) * H * d, d, static_cast<int64_t>(H) * d};
+  return {static_cast<int64_t>(H) * S * d, static_cast<int64_t>(S) * d, d};
+}
+
+// 4-D bf16 map (d, S, H, B) over a [B, H, S, d] tensor stored in `layout`;
+// box = {64, box_rows, 1, 1}, 128-byte swizzle, zero fill outside the tensor.
+bool make_map4(CUtensorMap* map, const void* base, int layout, int B, int H, int S, int d, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const Strides st = layout_strides(layout, H, S, d);
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(st.r) * 2, static_cast<cuuint64_t>(st.h) * 2,
+                                 static_cast<cuuint64_t>(st.b) * 2};
+  const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -290,9 +317,11 @@ attn_status_t launch_decode(const DecodeParams& prm, int grid, float* part_o, fl
   ccfg.stream = st;
   ccfg.attrs = attr;
   ccfg.numAttrs = 1;
+  // q and o share the layout (q's strides are the caller's choice of layout)
+  const RowLayout ol = {prm.Hq, prm.Sq, prm.q_sb, prm.q_sh, prm.q_sr};
   return cudaLaunchKernelEx(&ccfg, decode_combine_kernel<D>, static_cast<const float*>(part_o),
                             static_cast<const float2*>(part_ml), static_cast<uint16_t*>(o), lse, rows,
-                            prm.nsplit) == cudaSuccess
+                            prm.nsplit, ol) == cudaSuccess
              ? ATTN_OK
              : ATTN_ERR_CUDA;
 }
@@ -323,11 +352,16 @@ static attn_status_t fwd_impl(const void* q, const void* k, const void* v, const
   const float sc = effective_scale(scale, d);
   PrefillParams prm;
   std::memset(&prm, 0, sizeof(prm));
-  if (!make_map(&prm.tm_q, q, d, Sq, static_cast<int64_t>(B) * Hq, kBlockM) ||
-      !make_map(&prm.tm_k, k, d, Sk, static_cast<int64_t>(B) * Hkv, kBlockN) ||
-      !make_map(&prm.tm_v, v, d, Sk, static_cast<int64_t>(B) * Hkv, kBlockN))
+  const int layout = ex ? ex->layout : ATTN_LAYOUT_BHSD;
+  if (!make_map4(&prm.tm_q, q, layout, B, Hq, Sq, d, kBlockM) ||
+      !make_map4(&prm.tm_k, k, layout, B, Hkv, Sk, d, kBlockN) ||
+      !make_map4(&prm.tm_v, v, layout, B, Hkv, Sk, d, kBlockN))
     return ATTN_ERR_CUDA;
   prm.o = static_cast<uint16_t*>(o);
+  const Strides os = layout_strides(layout, Hq, Sq, d);
+  prm.o_sb = os.b;
+  prm.o_sh = os.h;
+  prm.o_sr = os.r;
   prm.lse = lse;
   prm.seqlens_q = ex ? ex->seqlens_q : nullptr;
   prm.seqlens_k = ex ? ex->seqlens_k : nullptr;
@@ -432,6 +466,11 @@ static attn_status_t decode_impl(const void* q, const void* k_cache, const void*
   float* part_o = static_cast<float*>(workspace);
   float2* part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + rows * ns * d * sizeof(float));
   prm.q = static_cast<const uint16_t*>(q);
+  const int layout = ex ? ex->layout : ATTN_LAYOUT_BHSD;
+  const Strides qs = layout_strides(layout, Hq, Sq, d);
+  prm.q_sb = qs.b;
+  prm.q_sh = qs.h;
+  prm.q_sr = qs.r;
   prm.seqlens_k = seqlens_k;
   if (ex != nullptr && ex->bias != nullptr) {
     prm.bias = static_cast<const uint16_t*>(ex->bias);

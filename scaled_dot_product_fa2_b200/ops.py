@@ -13,6 +13,7 @@ import torch
 from . import _lib
 
 CAUSAL_NONE, CAUSAL_TOP_LEFT, CAUSAL_BOTTOM_RIGHT = 0, 1, 2
+LAYOUT_BHSD, LAYOUT_BSHD = 0, 1
 
 
 def _stream_handle(device: torch.device) -> int:
@@ -32,12 +33,20 @@ def _check_tensor(name: str, t: torch.Tensor, dtype: torch.dtype, ndim: int) -> 
         raise ValueError(f"{name} must be contiguous")
 
 
-def _shapes(q, k, v):
+def _shapes(q, k, v, q_layout=LAYOUT_BHSD, kv_layout=LAYOUT_BHSD):
+    """(B, Hq, Hkv, Sq, Sk, d) of q [B,Hq,Sq,d] (or [B,Sq,Hq,d] for BSHD) and
+    k, v [B,Hkv,Sk,d] (or [B,Sk,Hkv,d])."""
     _check_tensor("q", q, torch.bfloat16, 4)
     _check_tensor("k", k, torch.bfloat16, 4)
     _check_tensor("v", v, torch.bfloat16, 4)
-    B, Hq, Sq, d = q.shape
-    Bk, Hkv, Sk, dk = k.shape
+    if q_layout == LAYOUT_BSHD:
+        B, Sq, Hq, d = q.shape
+    else:
+        B, Hq, Sq, d = q.shape
+    if kv_layout == LAYOUT_BSHD:
+        Bk, Sk, Hkv, dk = k.shape
+    else:
+        Bk, Hkv, Sk, dk = k.shape
     if Bk != B or dk != d or tuple(v.shape) != tuple(k.shape):
         raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
     if not (q.device == k.device == v.device):
@@ -45,8 +54,11 @@ def _shapes(q, k, v):
     return B, Hq, Hkv, Sq, Sk, d
 
 
-def _outputs(q, out, lse, want_lse):
-    B, Hq, Sq, d = q.shape
+def _outputs(q, out, lse, want_lse, layout=LAYOUT_BHSD):
+    if layout == LAYOUT_BSHD:
+        B, Sq, Hq, d = q.shape
+    else:
+        B, Hq, Sq, d = q.shape
     if out is None:
         out = torch.empty_like(q)
     else:
@@ -78,24 +90,26 @@ def _bias_extras(bias, B, Hq, Sq, Sk, device, ex=None):
 
 
 def attn_fwd(q, k, v, causal: int = CAUSAL_NONE, scale: float = 0.0, out=None, lse=None,
-             return_lse: bool = True, bias=None):
+             return_lse: bool = True, bias=None, layout: int = LAYOUT_BHSD):
     """O = softmax(scale * q k^T + bias + mask) v through the C ABI.
 
-    q [B,Hq,Sq,d], k/v [B,Hkv,Sk,d] bf16 contiguous CUDA tensors; ``scale=0``
-    means 1/sqrt(d); ``bias`` an optional bf16 [1|B, 1|Hq, Sq, Sk] tensor
-    (``attn_fwd_ex``).  Returns (o, lse) with lse fp32 [B,Hq,Sq] (None when
+    q [B,Hq,Sq,d], k/v [B,Hkv,Sk,d] bf16 contiguous CUDA tensors ([B,S,H,d]
+    for all four with ``layout=LAYOUT_BSHD``); ``scale=0`` means 1/sqrt(d);
+    ``bias`` an optional bf16 [1|B, 1|Hq, Sq, Sk] tensor (``attn_fwd_ex``).
+    Returns (o, lse) with o shaped like q and lse fp32 [B,Hq,Sq] (None when
     ``return_lse`` is False and no ``lse`` buffer was given).
     """
-    B, Hq, Hkv, Sq, Sk, d = _shapes(q, k, v)
-    out, lse = _outputs(q, out, lse, return_lse)
+    B, Hq, Hkv, Sq, Sk, d = _shapes(q, k, v, layout, layout)
+    out, lse = _outputs(q, out, lse, return_lse, layout)
     lib = _lib.get()
     with torch.cuda.device(q.device):
         args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr() if lse is not None else None,
                 B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal))
-        if bias is None:
+        if bias is None and layout == LAYOUT_BHSD:
             st = lib.attn_fwd(*args, _stream_handle(q.device))
         else:
             ex = _bias_extras(bias, B, Hq, Sq, Sk, q.device)
+            ex.layout = int(layout)
             st = lib.attn_fwd_ex(*args, ctypes.byref(ex), _stream_handle(q.device))
     _lib.check(st, "attn_fwd")
     return out, lse
@@ -150,13 +164,14 @@ def decode_workspace(q, k_cache, num_splits: int = 0) -> torch.Tensor:
 
 def attn_decode_splitkv(q, k_cache, v_cache, causal: int = CAUSAL_BOTTOM_RIGHT, scale: float = 0.0,
                         num_splits: int = 0, workspace=None, out=None, lse=None, return_lse: bool = True,
-                        bias=None, seqlens_k=None):
+                        bias=None, seqlens_k=None, layout: int = LAYOUT_BHSD):
     """Split-KV decode through the C ABI (``attn_decode_splitkv``, or
-    ``attn_decode_splitkv_ex`` when a bf16 ``bias`` [1|B, 1|Hq, Sq, Sk] or
-    int32 ``seqlens_k`` [B] is given).  Returns (o, lse)."""
-    if bias is not None or seqlens_k is not None:
+    ``attn_decode_splitkv_ex`` when a bf16 ``bias`` [1|B, 1|Hq, Sq, Sk], an
+    int32 ``seqlens_k`` [B] or ``layout=LAYOUT_BSHD`` (q and o as [B,Sq,Hq,d];
+    the cache stays [B,Hkv,Sk,d]) is given).  Returns (o, lse)."""
+    if bias is not None or seqlens_k is not None or layout != LAYOUT_BHSD:
         return _decode_ex(q, k_cache, v_cache, causal, scale, num_splits, workspace, out, lse, return_lse, bias,
-                          seqlens_k)
+                          seqlens_k, layout)
     B, Hq, Hkv, Sq, Sk, d = _shapes(q, k_cache, v_cache)
     out, lse = _outputs(q, out, lse, return_lse)
     if workspace is None:
@@ -174,15 +189,19 @@ def attn_decode_splitkv(q, k_cache, v_cache, causal: int = CAUSAL_BOTTOM_RIGHT, 
     return out, lse
 
 
-def _decode_ex(q, k_cache, v_cache, causal, scale, num_splits, workspace, out, lse, return_lse, bias, seqlens_k):
-    B, Hq, Hkv, Sq, Sk, d = _shapes(q, k_cache, v_cache)
+def _decode_ex(q, k_cache, v_cache, causal, scale, num_splits, workspace, out, lse, return_lse, bias, seqlens_k,
+               layout=LAYOUT_BHSD):
+    B, Hq, Hkv, Sq, Sk, d = _shapes(q, k_cache, v_cache, layout, LAYOUT_BHSD)
     ex = _bias_extras(bias, B, Hq, Sq, Sk, q.device)
+    ex.layout = int(layout)
     if seqlens_k is not None:
         _check_lengths("seqlens_k", seqlens_k, B, q.device)
         ex.seqlens_k = seqlens_k.data_ptr()
-    out, lse = _outputs(q, out, lse, return_lse)
+    out, lse = _outputs(q, out, lse, return_lse, layout)
     if workspace is None:
-        workspace = decode_workspace(q, k_cache, num_splits)
+        with torch.cuda.device(q.device):
+            n = decode_workspace_size(B, Hq, Hkv, Sq, Sk, d, num_splits)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
     if workspace.device != q.device or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous buffer on q's device")
     lib = _lib.get()

@@ -145,6 +145,9 @@ def test_extras_are_validated_on_host(lib):
     ex2 = Extras()
     ex2.seqlens_q = P
     assert dec(ex2) == 2             # the decode takes no query lengths
+    ex3 = Extras()
+    ex3.layout = 2
+    assert dec(ex3) == 2             # unknown layout
 
 
 def test_ptxas_report_checker():
