@@ -20,6 +20,9 @@ Sources followed (page title and section):
   * same page, same section: additive attention bias applied with the causal
     mask, two leading dims broadcasting over batch and heads
       -> attn_fwd(..., bias=...), attn_rows(..., bias=...)
+  * same page, section 2: the fused split of a packed QKV projection with
+    rotary embedding and copy into the KV cache (plain numpy, fp64)
+      -> rope_append
 """
 from __future__ import annotations
 
@@ -209,3 +212,49 @@ def split_combine(part_o, part_m, part_l):
     if st != 0:
         raise ValueError(f"oracle_split_combine failed ({st})")
     return o, lse
+
+
+# --------------------------------------------------------- rotary + KV append
+
+def rope_append(packed_qkv, cos, sin, past_lens, k_cache, v_cache, Hq: int, Hkv: int):
+    """The step before the decode, in plain fp64 loops: split a packed
+    [B, S_new, (Hq + 2*Hkv) * d] projection into q, k, v heads (q heads first,
+    then k, then v), rotate q and k by their absolute position, and append k, v
+    to the caches at rows past_lens[b] .. past_lens[b] + S_new - 1.
+
+    Follows the fused "split packed QKV with rotary embedding and copy KV" step
+    named by "[onnxruntime] WebGPU FlashAttention: kernel fusion and variable
+    sequence length" (section 2).  The page gives no formula; reading taken:
+    the non-interleaved rotary embedding -- for position p and i < d/2,
+    (x_i, x_{i+d/2}) -> (x_i cos[p,i] - x_{i+d/2} sin[p,i],
+                         x_{i+d/2} cos[p,i] + x_i sin[p,i]).
+    Returns (q [B, Hq, S_new, d], new k_cache, new v_cache [B, Hkv, cap, d],
+    total_lens [B] = past_lens + S_new).  Inputs are not modified.
+    """
+    x = _f64(packed_qkv)
+    cos, sin = _f64(cos), _f64(sin)
+    kc, vc = _f64(k_cache).copy(), _f64(v_cache).copy()
+    past = [int(p) for p in np.asarray(past_lens).reshape(-1)]
+    B, S_new, width = x.shape
+    d = width // (Hq + 2 * Hkv)
+    half = d // 2
+    q = np.zeros((B, Hq, S_new, d))
+
+    def rotate(vec, pos):
+        out = np.empty(d)
+        for i in range(half):
+            c, s = cos[pos, i], sin[pos, i]
+            out[i] = vec[i] * c - vec[i + half] * s
+            out[i + half] = vec[i + half] * c + vec[i] * s
+        return out
+
+    for b in range(B):
+        for s in range(S_new):
+            pos = past[b] + s
+            row = x[b, s]
+            for h in range(Hq):
+                q[b, h, s] = rotate(row[h * d:(h + 1) * d], pos)
+            for h in range(Hkv):
+                kc[b, h, pos] = rotate(row[(Hq + h) * d:(Hq + h + 1) * d], pos)
+                vc[b, h, pos] = row[(Hq + Hkv + h) * d:(Hq + Hkv + h + 1) * d]
+    return q, kc, vc, np.asarray([p + S_new for p in past], dtype=np.int64)

@@ -406,3 +406,81 @@ def test_bias_rows_api_matches_full(oracle_mod):
     o_r, l_r = oracle_mod.attn_rows(q, k, v, 0.5, TL, rows, bias=bias)
     assert np.allclose(o_r, o.reshape(-1, d)[rows], atol=1e-13)
     assert np.allclose(l_r, lse.reshape(-1)[rows], atol=1e-13)
+
+
+# ------------------------------------------------------ rotary + KV append
+# (the fused split / rotary / copy-KV step named by the decode page, section 2;
+# reading: non-interleaved rotary embedding)
+
+def _rope_tables(max_pos, d, base=10000.0):
+    inv = base ** (-np.arange(0, d // 2) * 2.0 / d)
+    ang = np.arange(max_pos)[:, None] * inv[None, :]
+    return np.cos(ang), np.sin(ang)
+
+
+def test_rope_relative_position_property(oracle_mod):
+    """RoPE's defining property: the rotated q.k depends only on the distance
+    between the two positions (shifting both positions leaves it unchanged),
+    and equals the plain q.k at distance 0."""
+    d, cap = 8, 64
+    cos, sin = _rope_tables(cap, d)
+    rng = np.random.default_rng(20)
+    qv, kv = rng.standard_normal(d), rng.standard_normal(d)
+
+    def rotated_dot(pq, pk):
+        packed_q = np.zeros((1, 1, 3 * d))
+        packed_q[0, 0, :d] = qv
+        packed_q[0, 0, d:2 * d] = kv
+        qa, ka, _, _ = oracle_mod.rope_append(packed_q, cos, sin, [pq], np.zeros((1, 1, cap, d)),
+                                              np.zeros((1, 1, cap, d)), 1, 1)
+        packed_k = packed_q.copy()
+        _, kb, _, _ = oracle_mod.rope_append(packed_k, cos, sin, [pk], np.zeros((1, 1, cap, d)),
+                                             np.zeros((1, 1, cap, d)), 1, 1)
+        return float(qa[0, 0, 0] @ kb[0, 0, pk])
+
+    assert abs(rotated_dot(5, 5) - float(qv @ kv)) < 1e-12
+    for dist in (0, 1, 3, 7):
+        ref = rotated_dot(10 + dist, 10)
+        for shift in (0, 4, 20):
+            assert abs(rotated_dot(10 + dist + shift, 10 + shift) - ref) < 1e-10
+    # and it does change with distance (the rotation is not the identity)
+    assert abs(rotated_dot(13, 10) - rotated_dot(10, 10)) > 1e-3
+
+
+def test_rope_append_positions_norms_and_untouched_rows(oracle_mod):
+    """Position 0 is the identity; every (i, i + d/2) pair keeps its norm;
+    v rows are copied unrotated to rows past .. past + S_new - 1, the other
+    cache rows are unchanged, and the total lengths are past + S_new."""
+    B, S_new, Hq, Hkv, d, cap = 2, 3, 4, 2, 8, 16
+    cos, sin = _rope_tables(cap, d)
+    rng = np.random.default_rng(21)
+    packed = rng.standard_normal((B, S_new, (Hq + 2 * Hkv) * d))
+    kc0, vc0 = rng.standard_normal((B, Hkv, cap, d)), rng.standard_normal((B, Hkv, cap, d))
+    past = [0, 9]
+    q, kc, vc, tot = oracle_mod.rope_append(packed, cos, sin, past, kc0, vc0, Hq, Hkv)
+    assert list(tot) == [3, 12]
+    half = d // 2
+    # batch 0, token 0 sits at position 0: no rotation
+    assert np.allclose(q[0, :, 0], packed[0, 0, :Hq * d].reshape(Hq, d), atol=0)
+    for b in range(B):
+        for s in range(S_new):
+            pos = past[b] + s
+            for h in range(Hq):
+                x = packed[b, s, h * d:(h + 1) * d]
+                y = q[b, h, s]
+                assert np.allclose(np.hypot(y[:half], y[half:]), np.hypot(x[:half], x[half:]), atol=1e-12)
+            for h in range(Hkv):
+                assert np.array_equal(vc[b, h, pos], packed[b, s, (Hq + Hkv + h) * d:(Hq + Hkv + h + 1) * d])
+        rows = [r for r in range(cap) if not past[b] <= r < past[b] + S_new]
+        assert np.array_equal(kc[b][:, rows], kc0[b][:, rows]) and np.array_equal(vc[b][:, rows], vc0[b][:, rows])
+
+
+def test_rope_quarter_turn_closed_form(oracle_mod):
+    """With cos = 0, sin = 1 (a quarter turn) the pair (a, b) becomes (-b, a)."""
+    d, cap = 4, 2
+    cos, sin = np.zeros((cap, d // 2)), np.ones((cap, d // 2))
+    packed = np.arange(1, 3 * d + 1, dtype=float).reshape(1, 1, 3 * d)
+    q, kc, _, _ = oracle_mod.rope_append(packed, cos, sin, [1], np.zeros((1, 1, cap, d)),
+                                         np.zeros((1, 1, cap, d)), 1, 1)
+    assert np.array_equal(q[0, 0, 0], np.array([-3.0, -4.0, 1.0, 2.0]))
+    assert np.array_equal(kc[0, 0, 1], np.array([-7.0, -8.0, 5.0, 6.0]))
