@@ -330,6 +330,27 @@ class GpuDecodeVarlen(GpuDecode):
         return kv + 2 * w.B * w.Hq * w.Sq * w.d * 2 + w.B * w.Hq * w.Sq * 4
 
 
+class GpuRopeAppend:
+    """The step before a decode: split the packed QKV, rotate q and k, append
+    k and v to the cache (one launch of the rotary/append kernel)."""
+
+    def __init__(self, w, rank: int):
+        self.w = w
+        past = [0] * w.B if w.Sq > 1 else None
+        packed, kc, vc, past_lens = inputs.make_rope_inputs(w.B, w.Sq, w.Hq, w.Hkv, w.d, w.Sk,
+                                                            w.seed + 7919 * rank, past_lens=past)
+        cos, sin = inputs.rope_tables(w.Sk, w.d)
+        self.packed, self.kc, self.vc = packed.cuda(), kc.cuda(), vc.cuda()
+        self.cos, self.sin, self.past = cos.cuda(), sin.cuda(), past_lens.cuda()
+        self.q = torch.empty((w.B, w.Hq, w.Sq, w.d), dtype=torch.bfloat16, device="cuda")
+        self.tot = torch.empty(w.B, dtype=torch.int32, device="cuda")
+
+    def run(self):
+        import scaled_dot_product_fa2_b200 as sdpa
+        sdpa.attn_rope_append(self.packed, self.cos, self.sin, self.past, self.kc, self.vc, self.w.Hq, self.w.Hkv,
+                              q_out=self.q, total_lens=self.tot)
+
+
 def timed_calls(fns, flush, reps: int, warmup: int):
     """Per-call CUDA-event times (ms) on the current stream, L2 flushed before each call."""
     stream = torch.cuda.current_stream()
@@ -551,6 +572,24 @@ def measure_breakdown(flush, peak_tf, hbm_gbs, rank, reps: int = 10):
         out[w.name + "_varlen"] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4),
                                    "lengths": s.lens, "launches_per_call": 2}
         del s
+    # rotary/append over a 4096-token prompt: 805 MB moved per call (> L2), no flush needed
+    s = GpuRopeAppend(inputs.ROPE_PROMPT, rank)
+    ms = statistics.median(timed_calls([s.run], slack_only, reps, 3)[0])
+    gbs = inputs.rope_bytes(s.w) / ms / 1e6
+    out[s.w.name] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4),
+                     "launches_per_call": 1}
+    del s
+    # one new token per sequence: 393 KB per call, a latency figure (L2-resident)
+    s = GpuRopeAppend(inputs.ROPE_DECODE, rank)
+
+    def batch(s=s):
+        for _ in range(DECODE_BATCH):
+            s.run()
+
+    ms = statistics.median(timed_calls([batch], slack_only, reps, 2)[0]) / DECODE_BATCH
+    out[s.w.name] = {"ms": round(ms, 4), "gbs": round(inputs.rope_bytes(s.w) / ms / 1e6, 1),
+                     "launches_per_call": 1}
+    del s
     torch.cuda.empty_cache()
     return out
 
@@ -559,9 +598,14 @@ def run_profile_case(args):
     """A few back-to-back calls of one workload with an L2 flush before each:
     the small, self-terminating command that ncu captures are taken on."""
     import scaled_dot_product_fa2_b200 as sdpa
-    w = inputs.BY_NAME[args.profile]
+    rope = {inputs.ROPE_PROMPT.name: inputs.ROPE_PROMPT, inputs.ROPE_DECODE.name: inputs.ROPE_DECODE}
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    runner = GpuDecode(w, 0) if w.decode else GpuPrefill(w, 0)
+    if args.profile in rope:
+        w = rope[args.profile]
+        runner = GpuRopeAppend(w, 0)
+    else:
+        w = inputs.BY_NAME[args.profile]
+        runner = GpuDecode(w, 0) if w.decode else GpuPrefill(w, 0)
     for _ in range(args.profile_calls):
         flush_buf.fill_(1)
         torch.cuda._sleep(HOST_SLACK_CYCLES)

@@ -71,7 +71,8 @@ typedef enum {
   ATTN_ERR_SCRATCH_LIMIT = 12, /* attn_decode_splitkv_static: problem needs more than
                                   ATTN_STATIC_SCRATCH_BYTES of scratch */
   ATTN_ERR_SEQLEN = 13         /* reported by attn_check_device_error: a per-batch length read on
-                                  the device was outside its valid range and was clamped */
+                                  the device was outside its valid range and was clamped, or a
+                                  position of attn_rope_append was out of range and skipped */
 } attn_status_t;
 
 enum { ATTN_CAUSAL_NONE = 0, ATTN_CAUSAL_TOP_LEFT = 1, ATTN_CAUSAL_BOTTOM_RIGHT = 2 };
@@ -263,6 +264,45 @@ attn_status_t attn_decode_splitkv_static(const void* q, const void* k_cache, con
                                          float* lse, int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale,
                                          int causal, int num_splits, void* stream);
 
+/*
+ * The step before a decode: split a packed QKV projection, rotate q and k by
+ * the rotary embedding, append k and v to the KV cache -- one streaming kernel.
+ * This is the fused "split packed QKV with rotary embedding and copy KV" step
+ * of "[onnxruntime] WebGPU FlashAttention: kernel fusion and variable sequence
+ * length" (section 2).  The page names the step but gives no formula; this
+ * library takes the non-interleaved rotary embedding: for position p and
+ * i < d/2 the pair (x_i, x_{i+d/2}) becomes
+ *   (x_i cos[p][i] - x_{i+d/2} sin[p][i],  x_{i+d/2} cos[p][i] + x_i sin[p][i]),
+ * computed in fp32 and rounded once to bf16.  Token t of batch b sits at the
+ * absolute position p = past_lens[b] + t.
+ *
+ *   packed_qkv  [B, S_new, (Hq + 2*Hkv) * d] bf16, device; each token's row
+ *               holds Hq q heads, then Hkv k heads, then Hkv v heads, d each.
+ *   cos_table,
+ *   sin_table   [max_pos, d/2] fp32, device (the caller picks the frequencies).
+ *   past_lens   [B] int32, device: tokens already in the cache per batch.
+ *   q_out       rotated q, [B, Hq, S_new, d] bf16 (layout BSHD: [B, S_new, Hq, d]).
+ *   k_cache,
+ *   v_cache     [B, Hkv, cap, d] bf16 (layout BSHD: [B, cap, Hkv, d]), device,
+ *               updated in place: rows past_lens[b] .. past_lens[b] + S_new - 1
+ *               receive the rotated k and the unchanged v; no other row is touched.
+ *   total_lens  [B] int32, device, or NULL: receives past_lens[b] + S_new, the
+ *               key lengths for attn_decode_splitkv_varlen over the updated cache.
+ *   layout      ATTN_LAYOUT_BHSD or ATTN_LAYOUT_BSHD, for q_out and both caches.
+ *
+ * All buffers are the caller's; the library allocates nothing.  Pointers must
+ * be 16-byte aligned (past_lens, total_lens: 4 bytes).  Host-side errors:
+ * ATTN_ERR_SHAPE (negative size, cap or max_pos < 1, unknown layout),
+ * ATTN_ERR_GQA, ATTN_ERR_HEADDIM (d not 64 or 128), ATTN_ERR_NULL,
+ * ATTN_ERR_ALIGN.  B == 0 or S_new == 0 writes only total_lens.  A token whose
+ * position falls outside [0, min(cap, max_pos)) is skipped (nothing of its row
+ * is written) and attn_check_device_error() then returns ATTN_ERR_SEQLEN.
+ * Asynchronous on `stream`.
+ */
+attn_status_t attn_rope_append(const void* packed_qkv, const float* cos_table, const float* sin_table, int max_pos,
+                               const int* past_lens, void* q_out, void* k_cache, void* v_cache, int* total_lens,
+                               int B, int S_new, int Hq, int Hkv, int cap, int d, int layout, void* stream);
+
 /* A static, human-readable name for a status code. */
 const char* attn_status_string(attn_status_t status);
 
@@ -270,7 +310,8 @@ const char* attn_status_string(attn_status_t status);
  * Synchronizes `stream`, then reads and clears the device error word.
  * Returns ATTN_ERR_DEVICE_TIMEOUT if a kernel gave up on a bounded wait since
  * the last check, else ATTN_ERR_SEQLEN if attn_fwd_varlen or
- * attn_decode_splitkv_varlen had to clamp a per-batch length, ATTN_ERR_CUDA
+ * attn_decode_splitkv_varlen had to clamp a per-batch length or
+ * attn_rope_append skipped a token, ATTN_ERR_CUDA
  * if the synchronization itself failed, else ATTN_OK.
  */
 attn_status_t attn_check_device_error(void* stream);

@@ -14,6 +14,7 @@
 #include "sdpa_b200.h"
 #include "decode.cuh"
 #include "prefill.cuh"
+#include "rope.cuh"
 
 namespace sdpa {
 constexpr int kMaxDeviceSlots = 64;
@@ -326,6 +327,18 @@ attn_status_t launch_decode(const DecodeParams& prm, int grid, float* part_o, fl
              : ATTN_ERR_CUDA;
 }
 
+// Blocks for the rotary/append kernel: enough rows for every lane, at most one
+// resident wave (kRopeBlocksPerSm per SM); the kernel strides over the rest.
+template <int D>
+attn_status_t launch_rope(const RopeParams& prm, int sms, cudaStream_t st) {
+  constexpr int kRowsPerBlock = kRopeWarps * (32 / (D / 8)) * kRopeUnroll;
+  const int64_t need = std::max<int64_t>(1, (prm.rows + kRowsPerBlock - 1) / kRowsPerBlock);
+  const int64_t wave = static_cast<int64_t>(sms) * kRopeBlocksPerSm;
+  const int grid = static_cast<int>(std::min(need, wave));
+  rope_append_kernel<D><<<grid, kRopeWarps * 32, 0, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace sdpa
 
@@ -528,6 +541,60 @@ attn_status_t attn_decode_splitkv_ex(const void* q, const void* k_cache, const v
                      workspace, workspace_bytes, stream);
 }
 
+attn_status_t attn_rope_append(const void* packed_qkv, const float* cos_table, const float* sin_table, int max_pos,
+                               const int* past_lens, void* q_out, void* k_cache, void* v_cache, int* total_lens,
+                               int B, int S_new, int Hq, int Hkv, int cap, int d, int layout, void* stream) {
+  if (B < 0 || S_new < 0 || Hq <= 0 || Hkv <= 0 || cap <= 0 || max_pos <= 0) return ATTN_ERR_SHAPE;
+  if (S_new > kMaxSeq || cap > kMaxSeq || max_pos > kMaxSeq) return ATTN_ERR_SHAPE;
+  if (static_cast<int64_t>(B) * (Hq + 2 * static_cast<int64_t>(Hkv)) > INT_MAX / 4) return ATTN_ERR_SHAPE;
+  if (Hq % Hkv != 0) return ATTN_ERR_GQA;
+  if (d != 64 && d != 128) return ATTN_ERR_HEADDIM;
+  if (layout != ATTN_LAYOUT_BHSD && layout != ATTN_LAYOUT_BSHD) return ATTN_ERR_SHAPE;
+  if (B == 0) return ATTN_OK;
+  if (past_lens == nullptr) return ATTN_ERR_NULL;
+  if (!aligned(past_lens, 4) || (total_lens != nullptr && !aligned(total_lens, 4))) return ATTN_ERR_ALIGN;
+  if (S_new > 0) {
+    if (packed_qkv == nullptr || cos_table == nullptr || sin_table == nullptr || q_out == nullptr ||
+        k_cache == nullptr || v_cache == nullptr)
+      return ATTN_ERR_NULL;
+    if (!aligned(packed_qkv, 16) || !aligned(cos_table, 16) || !aligned(sin_table, 16) || !aligned(q_out, 16) ||
+        !aligned(k_cache, 16) || !aligned(v_cache, 16))
+      return ATTN_ERR_ALIGN;
+  } else if (total_lens == nullptr) {
+    return ATTN_OK;  // nothing to write
+  }
+  int dev = 0, sms = 0;
+  attn_status_t s = current_device(&dev, &sms);
+  if (s != ATTN_OK) return s;
+  RopeParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.packed = static_cast<const uint16_t*>(packed_qkv);
+  prm.cos_t = cos_table;
+  prm.sin_t = sin_table;
+  prm.past_lens = past_lens;
+  prm.q_out = static_cast<uint16_t*>(q_out);
+  prm.k_cache = static_cast<uint16_t*>(k_cache);
+  prm.v_cache = static_cast<uint16_t*>(v_cache);
+  prm.total_lens = total_lens;
+  const Strides qs = layout_strides(layout, Hq, S_new, d);
+  const Strides cs = layout_strides(layout, Hkv, cap, d);
+  prm.q_sb = qs.b;
+  prm.q_sh = qs.h;
+  prm.q_sr = qs.r;
+  prm.c_sb = cs.b;
+  prm.c_sh = cs.h;
+  prm.c_sr = cs.r;
+  prm.rows = static_cast<int64_t>(B) * S_new * (Hq + 2 * Hkv);
+  prm.B = B;
+  prm.S_new = S_new;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.cap = cap;
+  prm.max_pos = max_pos;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 128 ? launch_rope<128>(prm, sms, st) : launch_rope<64>(prm, sms, st);
+}
+
 const char* attn_status_string(attn_status_t status) {
   switch (status) {
     case ATTN_OK: return "ok";
@@ -543,7 +610,7 @@ const char* attn_status_string(attn_status_t status) {
     case ATTN_ERR_ARCH: return "the current device is not sm_100 (B200)";
     case ATTN_ERR_SCALE: return "scale must be 0 (default) or finite and > 0";
     case ATTN_ERR_SCRATCH_LIMIT: return "problem needs more than the library's static decode scratch (16 MiB)";
-    case ATTN_ERR_SEQLEN: return "a per-batch key length was outside [0, cache capacity] (clamped)";
+    case ATTN_ERR_SEQLEN: return "a per-batch length or position was outside its range (clamped or skipped)";
   }
   return "unknown status";
 }

@@ -131,3 +131,55 @@ def prefill_lengths(w: Workload) -> list[int]:
     lens = torch.randint(w.Sq // 8, w.Sq + 1, (w.B,), generator=g, dtype=torch.int64).tolist()
     lens[0] = w.Sq
     return [int(x) for x in lens]
+
+
+#: the step before a decode: split a packed QKV of one new token per sequence,
+#: rotate q and k, append k and v to a cache of 8192 rows (the decode's shape)
+ROPE_DECODE = Workload("rope_append_decode_b8_hq32_hkv8", B=8, Hq=32, Hkv=8, Sq=1, Sk=8192, d=128,
+                       causal=CAUSAL_NONE, seed=7000)
+#: the same step over a whole 4096-token prompt (the prefill's shape), into an
+#: empty cache of 4096 rows
+ROPE_PROMPT = Workload("rope_append_prompt_b8_s4096_h16", B=8, Hq=16, Hkv=16, Sq=4096, Sk=4096, d=128,
+                       causal=CAUSAL_NONE, seed=7001)
+
+
+def rope_bytes(w: Workload) -> int:
+    """Algorithmic bytes of one rotary/append call: the packed projection read
+    once, q written once, k and v written once into the cache (bf16).  The
+    cos/sin rows (4*d bytes a token, about 2% of the rest) are left out: they
+    are shared across sequences and heads and stay in L2."""
+    per_token = (w.Hq + 2 * w.Hkv) * w.d * 2
+    return 2 * w.B * w.Sq * per_token
+
+
+def rope_tables(max_pos: int, d: int, base: float = 10000.0):
+    """cos/sin tables [max_pos, d/2] fp32 of the usual rotary frequencies:
+    angle(p, i) = p * base^(-2i/d), evaluated in fp64 and rounded to fp32.
+    The kernel and the oracle both take these tables as inputs."""
+    p = torch.arange(max_pos, dtype=torch.float64)[:, None]
+    i = torch.arange(d // 2, dtype=torch.float64)[None, :]
+    ang = p * torch.pow(torch.tensor(base, dtype=torch.float64), -2.0 * i / d)
+    return torch.cos(ang).float().contiguous(), torch.sin(ang).float().contiguous()
+
+
+def make_rope_inputs(B: int, S_new: int, Hq: int, Hkv: int, d: int, cap: int, seed: int,
+                     past_lens: list[int] | None = None, layout: int = 0):
+    """Seeded host tensors for the rotary/append step.
+
+    packed [B, S_new, (Hq+2*Hkv)*d], then k_cache and v_cache (their existing
+    contents; [B, Hkv, cap, d], or [B, cap, Hkv, d] for layout 1), all fp32
+    N(0, 1) from one CPU generator in that order and rounded to bf16; then,
+    unless given, past_lens uniform in [0, cap - S_new] from the same
+    generator with past_lens[0] = cap - S_new (a cache filled to capacity).
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    packed = torch.randn((B, S_new, (Hq + 2 * Hkv) * d), generator=g, dtype=torch.float32).bfloat16()
+    shape = (B, cap, Hkv, d) if layout == 1 else (B, Hkv, cap, d)
+    kc = torch.randn(shape, generator=g, dtype=torch.float32).bfloat16()
+    vc = torch.randn(shape, generator=g, dtype=torch.float32).bfloat16()
+    if past_lens is None:
+        past_lens = torch.randint(0, cap - S_new + 1, (B,), generator=g, dtype=torch.int64).tolist()
+        if B > 0:
+            past_lens[0] = cap - S_new
+    return packed, kc, vc, torch.tensor(past_lens, dtype=torch.int32)

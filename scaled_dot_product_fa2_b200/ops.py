@@ -264,6 +264,64 @@ def attn_decode_splitkv_static(q, k_cache, v_cache, causal: int = CAUSAL_BOTTOM_
     return out, lse
 
 
+def attn_rope_append(packed_qkv, cos, sin, past_lens, k_cache, v_cache, Hq: int, Hkv: int,
+                     layout: int = LAYOUT_BHSD, q_out=None, total_lens=None):
+    """Split a packed QKV projection, rotate q and k, append k and v to the cache
+    (``attn_rope_append``).
+
+    packed_qkv [B, S_new, (Hq + 2*Hkv) * d] bf16 (q heads, then k, then v);
+    cos, sin [max_pos, d/2] fp32; past_lens [B] int32; k_cache, v_cache
+    [B, Hkv, cap, d] bf16 ([B, cap, Hkv, d] for LAYOUT_BSHD), updated in place.
+    Returns (q [B, Hq, S_new, d] -- [B, S_new, Hq, d] for LAYOUT_BSHD --,
+    total_lens [B] int32 = past_lens + S_new).  A token whose position is out
+    of range is skipped and reported by check_device_error().
+    """
+    _check_tensor("packed_qkv", packed_qkv, torch.bfloat16, 3)
+    _check_tensor("k_cache", k_cache, torch.bfloat16, 4)
+    _check_tensor("v_cache", v_cache, torch.bfloat16, 4)
+    _check_tensor("cos", cos, torch.float32, 2)
+    _check_tensor("sin", sin, torch.float32, 2)
+    B, S_new, width = packed_qkv.shape
+    if Hq <= 0 or Hkv <= 0 or width % (Hq + 2 * Hkv) != 0:
+        raise ValueError("packed_qkv's last dim must be (Hq + 2*Hkv) * d")
+    d = width // (Hq + 2 * Hkv)
+    if layout == LAYOUT_BSHD:
+        cap = k_cache.shape[1]
+        cache_shape, q_shape = (B, cap, Hkv, d), (B, S_new, Hq, d)
+    elif layout == LAYOUT_BHSD:
+        cap = k_cache.shape[2]
+        cache_shape, q_shape = (B, Hkv, cap, d), (B, Hq, S_new, d)
+    else:
+        raise ValueError(f"unknown layout {layout}")
+    if tuple(k_cache.shape) != cache_shape or tuple(v_cache.shape) != cache_shape:
+        raise ValueError(f"k_cache and v_cache must be {cache_shape}")
+    if tuple(cos.shape) != tuple(sin.shape) or cos.shape[1] != d // 2:
+        raise ValueError("cos and sin must both be [max_pos, d/2]")
+    dev = packed_qkv.device
+    for name, t in (("k_cache", k_cache), ("v_cache", v_cache), ("cos", cos), ("sin", sin)):
+        if t.device != dev:
+            raise ValueError(f"{name} must be on packed_qkv's device")
+    _check_lengths("past_lens", past_lens, B, dev)
+    if q_out is None:
+        q_out = torch.empty(q_shape, dtype=torch.bfloat16, device=dev)
+    else:
+        _check_tensor("q_out", q_out, torch.bfloat16, 4)
+        if tuple(q_out.shape) != q_shape or q_out.device != dev:
+            raise ValueError(f"q_out must be {q_shape} on packed_qkv's device")
+    if total_lens is None:
+        total_lens = torch.empty(B, dtype=torch.int32, device=dev)
+    else:
+        _check_lengths("total_lens", total_lens, B, dev)
+    lib = _lib.get()
+    with torch.cuda.device(dev):
+        st = lib.attn_rope_append(packed_qkv.data_ptr(), cos.data_ptr(), sin.data_ptr(), int(cos.shape[0]),
+                                  past_lens.data_ptr(), q_out.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                  total_lens.data_ptr(), B, S_new, Hq, Hkv, cap, d, int(layout),
+                                  _stream_handle(dev))
+    _lib.check(st, "attn_rope_append")
+    return q_out, total_lens
+
+
 def check_device_error(device=None) -> None:
     """Synchronize the current stream and raise if a kernel gave up on a bounded wait."""
     dev = torch.device("cuda") if device is None else torch.device(device)

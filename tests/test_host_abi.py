@@ -186,3 +186,24 @@ def test_decode_split_policy_fills_one_wave(lib):
     # more pairs than resident slots: no splitting
     assert lib.attn_decode_num_splits(64, 32, 8, 1, 8192, 128) == 1
 
+
+
+def test_rope_append_rejects_bad_arguments_on_host(lib):
+    def call(packed=P, cos=P, sin=P, max_pos=64, past=P, q=P, kc=P, vc=P, tot=P, B=2, S_new=3, Hq=4, Hkv=2,
+             cap=64, d=128, layout=0):
+        return lib.attn_rope_append(packed, cos, sin, max_pos, past, q, kc, vc, tot, B, S_new, Hq, Hkv, cap, d,
+                                    layout, None)
+    for kw, status in [
+        (dict(packed=None), 1), (dict(cos=None), 1), (dict(sin=None), 1), (dict(past=None), 1),
+        (dict(q=None), 1), (dict(kc=None), 1), (dict(vc=None), 1),
+        (dict(B=-1), 2), (dict(S_new=-1), 2), (dict(Hq=0), 2), (dict(Hkv=0), 2), (dict(cap=0), 2),
+        (dict(max_pos=0), 2), (dict(layout=2), 2), (dict(S_new=(1 << 30) + 1), 2),
+        (dict(Hq=6, Hkv=4), 3),
+        (dict(d=96), 4), (dict(d=32), 4),
+        (dict(packed=P + 8), 5), (dict(cos=P + 4), 5), (dict(sin=P + 4), 5), (dict(q=P + 2), 5),
+        (dict(kc=P + 8), 5), (dict(vc=P + 8), 5), (dict(past=P + 2), 5), (dict(tot=P + 1), 5),
+    ]:
+        assert call(**kw) == status, kw
+    # nothing to do: no batch, or no new token and no total lengths wanted
+    assert call(B=0, packed=None, cos=None, sin=None, past=None, q=None, kc=None, vc=None, tot=None) == 0
+    assert call(S_new=0, packed=None, cos=None, sin=None, q=None, kc=None, vc=None, tot=None) == 0
