@@ -10,12 +10,15 @@
 // token t of batch b; k and v go to cache rows past_lens[b] .. + S_new - 1.
 //
 // A pure streaming kernel, bound by HBM bandwidth: every element of the packed
-// input is read once and written once (the cos/sin rows stay in L2).  One row
-// of d bf16 is held by d/8 lanes, 16 bytes each, so a warp covers 2 (d=128)
-// or 4 (d=64) rows per pass; the partner half of a rotated pair sits d/16
-// lanes away and comes over by shuffle.  Each lane keeps kRopeUnroll rows in
-// flight to cover HBM latency; the grid is a multiple of the SM count and
-// strides over the rows.
+// input is read once and written once (the cos/sin rows stay in L2).  A block
+// takes whole tokens (grid-stride over them), so the batch/token split and the
+// position check happen once per token and each lane loads its slice of the
+// token's cos/sin row once for all of the token's heads.  One row of d bf16 is
+// held by d/8 lanes, 16 bytes each: a warp covers 2 (d=128) or 4 (d=64) head
+// rows per pass, the block 8 times that, and every lane issues the loads of
+// kRopeUnroll passes before it uses any, to keep enough bytes in flight.  The
+// partner half of each rotated pair sits d/16 lanes away and comes over by
+// shuffle.
 #pragma once
 #include "ptx.cuh"
 
@@ -32,102 +35,93 @@ struct RopeParams {
   int* total_lens;         // [B] past + S_new, or nullptr
   int64_t q_sb, q_sh, q_sr;
   int64_t c_sb, c_sh, c_sr;
-  int64_t rows;            // B * S_new * (Hq + 2*Hkv)
+  int tokens;              // B * S_new (< 2^31, checked on the host)
   int B, S_new, Hq, Hkv, cap, max_pos;
 };
 
-constexpr int kRopeWarps = 8;   // warps per block (256 threads)
-constexpr int kRopeUnroll = 2;  // row groups per lane in flight
-constexpr int kRopeBlocksPerSm = 5;  // resident blocks per SM (48 registers a thread)
+constexpr int kRopeWarps = 8;        // warps per block (256 threads)
+constexpr int kRopeUnroll = 3;       // block passes over a token's head rows with loads in flight together
+constexpr int kRopeBlocksPerSm = 4;  // resident blocks per SM
 
 template <int D>
-__global__ void __launch_bounds__(kRopeWarps * 32, kRopeBlocksPerSm) rope_append_kernel(const __grid_constant__ RopeParams p) {
+__global__ void __launch_bounds__(kRopeWarps * 32, kRopeBlocksPerSm)
+    rope_append_kernel(const __grid_constant__ RopeParams p) {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   constexpr int kHalf = D / 2;
   constexpr int kLanesPerRow = D / 8;  // 16 bytes of the row per lane
   constexpr int kRowsPerPass = 32 / kLanesPerRow;
-  constexpr int kPartner = kLanesPerRow / 2;  // lane distance between x_i and x_{i+d/2}
+  constexpr int kBlockRows = kRopeWarps * kRowsPerPass;  // head rows per block pass
+  constexpr int kPartner = kLanesPerRow / 2;             // lane distance between x_i and x_{i+d/2}
   const int lane = threadIdx.x & 31;
   const int sub = lane % kLanesPerRow;
-  const bool first_half = sub < kPartner;
+  const int row_in_block = (threadIdx.x >> 5) * kRowsPerPass + lane / kLanesPerRow;
+  // the partner's element enters with a minus sign in the first half
+  // (x_i c - x_{i+d/2} s) and a plus sign in the second (x_{i+d/2} c + x_i s)
+  const float sign = sub < kPartner ? -1.f : 1.f;
   const int i0 = (sub % kPartner) * 8;  // index within the half of this lane's 8 elements
   const int slots = p.Hq + 2 * p.Hkv;
 
-  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (p.total_lens != nullptr && gtid < p.B) p.total_lens[gtid] = __ldg(p.past_lens + gtid) + p.S_new;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.B; i += gridDim.x * blockDim.x)
+    if (p.total_lens != nullptr) p.total_lens[i] = __ldg(p.past_lens + i) + p.S_new;
 
-  const int64_t warp = static_cast<int64_t>(blockIdx.x) * kRopeWarps + (threadIdx.x >> 5);
-  const int64_t step = static_cast<int64_t>(gridDim.x) * kRopeWarps * kRowsPerPass * kRopeUnroll;
-  for (int64_t base = warp * kRowsPerPass * kRopeUnroll; base < p.rows; base += step) {  // warp-uniform
-    uint4 x[kRopeUnroll];
-    uint16_t* dst[kRopeUnroll];
-    int kind[kRopeUnroll];  // 0: q, 1: k, 2: v, -1: nothing to write
-    int pos[kRopeUnroll];
-#pragma unroll
-    for (int u = 0; u < kRopeUnroll; ++u) {
-      const int64_t r = base + u * kRowsPerPass + lane / kLanesPerRow;
-      x[u] = make_uint4(0u, 0u, 0u, 0u);
-      kind[u] = -1;
-      pos[u] = 0;
-      dst[u] = nullptr;
-      if (r < p.rows) {
-        const int h = static_cast<int>(r % slots);
-        const int64_t bt = r / slots;
-        const int t = static_cast<int>(bt % p.S_new);
-        const int b = static_cast<int>(bt / p.S_new);
-        const int past = __ldg(p.past_lens + b);
-        const int ps = past + t;
-        if (past < 0 || ps >= p.cap || ps >= p.max_pos) {
-          if (sub == 0) atomicOr(&g_error_word, kErrSeqlen);
-        } else {
-          x[u] = __ldg(reinterpret_cast<const uint4*>(p.packed + r * D) + sub);
-          pos[u] = ps;
-          if (h < p.Hq) {
-            kind[u] = 0;
-            dst[u] = p.q_out + b * p.q_sb + h * p.q_sh + t * p.q_sr;
-          } else if (h < p.Hq + p.Hkv) {
-            kind[u] = 1;
-            dst[u] = p.k_cache + b * p.c_sb + (h - p.Hq) * p.c_sh + ps * p.c_sr;
-          } else {
-            kind[u] = 2;
-            dst[u] = p.v_cache + b * p.c_sb + (h - p.Hq - p.Hkv) * p.c_sh + ps * p.c_sr;
-          }
-        }
-      }
+  for (int bt = blockIdx.x; bt < p.tokens; bt += gridDim.x) {  // block-uniform
+    const int b = bt / p.S_new;
+    const int t = bt - b * p.S_new;
+    const int past = __ldg(p.past_lens + b);
+    const int pos = past + t;
+    if (past < 0 || pos >= p.cap || pos >= p.max_pos) {
+      if (threadIdx.x == 0) atomicOr(&g_error_word, kErrSeqlen);
+      continue;
     }
+    const float4* cr = reinterpret_cast<const float4*>(p.cos_t + static_cast<int64_t>(pos) * kHalf + i0);
+    const float4* sr = reinterpret_cast<const float4*>(p.sin_t + static_cast<int64_t>(pos) * kHalf + i0);
+    const float4 c0 = __ldg(cr), c1 = __ldg(cr + 1), s0 = __ldg(sr), s1 = __ldg(sr + 1);
+    const float c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    const float s[8] = {s0.x * sign, s0.y * sign, s0.z * sign, s0.w * sign,
+                        s1.x * sign, s1.y * sign, s1.z * sign, s1.w * sign};
+    const uint4* src = reinterpret_cast<const uint4*>(p.packed + static_cast<int64_t>(bt) * slots * D) + sub;
+    uint16_t* const q_base = p.q_out + b * p.q_sb + t * p.q_sr;
+    const int64_t c_off = b * p.c_sb + static_cast<int64_t>(pos) * p.c_sr;
+
+    for (int h0 = 0; h0 < slots; h0 += kBlockRows * kRopeUnroll) {  // block-uniform
+      uint4 x[kRopeUnroll];
 #pragma unroll
-    for (int u = 0; u < kRopeUnroll; ++u) {
-      // every lane of the warp takes part in the exchange; the partner lane
-      // always belongs to the same row
-      uint4 y;
-      y.x = __shfl_xor_sync(0xffffffffu, x[u].x, kPartner);
-      y.y = __shfl_xor_sync(0xffffffffu, x[u].y, kPartner);
-      y.z = __shfl_xor_sync(0xffffffffu, x[u].z, kPartner);
-      y.w = __shfl_xor_sync(0xffffffffu, x[u].w, kPartner);
-      if (kind[u] < 0) continue;
-      uint4 out = x[u];
-      if (kind[u] < 2) {
-        const float4* cr = reinterpret_cast<const float4*>(p.cos_t + static_cast<int64_t>(pos[u]) * kHalf + i0);
-        const float4* sr = reinterpret_cast<const float4*>(p.sin_t + static_cast<int64_t>(pos[u]) * kHalf + i0);
-        const float4 c0 = __ldg(cr), c1 = __ldg(cr + 1), s0 = __ldg(sr), s1 = __ldg(sr + 1);
-        const float c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const float s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-        const uint32_t xs[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
-        const uint32_t ys[4] = {y.x, y.y, y.z, y.w};
-        uint32_t o[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float xa = bf16_bits_to_float(static_cast<unsigned short>(xs[j] & 0xFFFFu));
-          const float xb = bf16_bits_to_float(static_cast<unsigned short>(xs[j] >> 16));
-          // the partner's element enters with a minus sign in the first half
-          // (x_i c - x_{i+d/2} s) and a plus sign in the second (x_{i+d/2} c + x_i s)
-          const float ya = bf16_bits_to_float(static_cast<unsigned short>(ys[j] & 0xFFFFu)) * (first_half ? -1.f : 1.f);
-          const float yb = bf16_bits_to_float(static_cast<unsigned short>(ys[j] >> 16)) * (first_half ? -1.f : 1.f);
-          o[j] = pack_bf16x2(fmaf(ya, s[2 * j], xa * c[2 * j]), fmaf(yb, s[2 * j + 1], xb * c[2 * j + 1]));
-        }
-        out = make_uint4(o[0], o[1], o[2], o[3]);
+      for (int u = 0; u < kRopeUnroll; ++u) {
+        const int h = h0 + u * kBlockRows + row_in_block;
+        x[u] = h < slots ? __ldg(src + h * (D / 8)) : make_uint4(0u, 0u, 0u, 0u);
       }
-      reinterpret_cast<uint4*>(dst[u])[sub] = out;
+#pragma unroll
+      for (int u = 0; u < kRopeUnroll; ++u) {
+        // every lane of the warp takes part in the exchange; the partner lane
+        // always belongs to the same row
+        uint4 y;
+        y.x = __shfl_xor_sync(0xffffffffu, x[u].x, kPartner);
+        y.y = __shfl_xor_sync(0xffffffffu, x[u].y, kPartner);
+        y.z = __shfl_xor_sync(0xffffffffu, x[u].z, kPartner);
+        y.w = __shfl_xor_sync(0xffffffffu, x[u].w, kPartner);
+        const int h = h0 + u * kBlockRows + row_in_block;
+        if (h >= slots) continue;
+        uint4 out = x[u];
+        uint16_t* dst;
+        if (h < p.Hq + p.Hkv) {
+          dst = h < p.Hq ? q_base + h * p.q_sh : p.k_cache + c_off + (h - p.Hq) * p.c_sh;
+          const uint32_t xs[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+          const uint32_t ys[4] = {y.x, y.y, y.z, y.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float xa = bf16_bits_to_float(static_cast<unsigned short>(xs[j] & 0xFFFFu));
+            const float xb = bf16_bits_to_float(static_cast<unsigned short>(xs[j] >> 16));
+            const float ya = bf16_bits_to_float(static_cast<unsigned short>(ys[j] & 0xFFFFu));
+            const float yb = bf16_bits_to_float(static_cast<unsigned short>(ys[j] >> 16));
+            o[j] = pack_bf16x2(fmaf(ya, s[2 * j], xa * c[2 * j]), fmaf(yb, s[2 * j + 1], xb * c[2 * j + 1]));
+          }
+          out = make_uint4(o[0], o[1], o[2], o[3]);
+        } else {
+          dst = p.v_cache + c_off + (h - p.Hq - p.Hkv) * p.c_sh;  // v: copied as is
+        }
+        reinterpret_cast<uint4*>(dst)[sub] = out;
+      }
     }
   }
 }

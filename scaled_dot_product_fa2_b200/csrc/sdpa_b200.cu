@@ -327,14 +327,12 @@ attn_status_t launch_decode(const DecodeParams& prm, int grid, float* part_o, fl
              : ATTN_ERR_CUDA;
 }
 
-// Blocks for the rotary/append kernel: enough rows for every lane, at most one
-// resident wave (kRopeBlocksPerSm per SM); the kernel strides over the rest.
+// Blocks for the rotary/append kernel: one per token, at most one resident
+// wave (kRopeBlocksPerSm per SM); the blocks stride over the remaining tokens.
 template <int D>
 attn_status_t launch_rope(const RopeParams& prm, int sms, cudaStream_t st) {
-  constexpr int kRowsPerBlock = kRopeWarps * (32 / (D / 8)) * kRopeUnroll;
-  const int64_t need = std::max<int64_t>(1, (prm.rows + kRowsPerBlock - 1) / kRowsPerBlock);
   const int64_t wave = static_cast<int64_t>(sms) * kRopeBlocksPerSm;
-  const int grid = static_cast<int>(std::min(need, wave));
+  const int grid = static_cast<int>(std::min<int64_t>(std::max(prm.tokens, 1), wave));
   rope_append_kernel<D><<<grid, kRopeWarps * 32, 0, st>>>(prm);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -547,6 +545,8 @@ attn_status_t attn_rope_append(const void* packed_qkv, const float* cos_table, c
   if (B < 0 || S_new < 0 || Hq <= 0 || Hkv <= 0 || cap <= 0 || max_pos <= 0) return ATTN_ERR_SHAPE;
   if (S_new > kMaxSeq || cap > kMaxSeq || max_pos > kMaxSeq) return ATTN_ERR_SHAPE;
   if (static_cast<int64_t>(B) * (Hq + 2 * static_cast<int64_t>(Hkv)) > INT_MAX / 4) return ATTN_ERR_SHAPE;
+  if (static_cast<int64_t>(B) * S_new > INT_MAX || Hq + 2 * static_cast<int64_t>(Hkv) > INT_MAX / 128)
+    return ATTN_ERR_SHAPE;
   if (Hq % Hkv != 0) return ATTN_ERR_GQA;
   if (d != 64 && d != 128) return ATTN_ERR_HEADDIM;
   if (layout != ATTN_LAYOUT_BHSD && layout != ATTN_LAYOUT_BSHD) return ATTN_ERR_SHAPE;
@@ -584,7 +584,7 @@ attn_status_t attn_rope_append(const void* packed_qkv, const float* cos_table, c
   prm.c_sb = cs.b;
   prm.c_sh = cs.h;
   prm.c_sr = cs.r;
-  prm.rows = static_cast<int64_t>(B) * S_new * (Hq + 2 * Hkv);
+  prm.tokens = B * S_new;
   prm.B = B;
   prm.S_new = S_new;
   prm.Hq = Hq;

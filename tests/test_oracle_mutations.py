@@ -75,3 +75,48 @@ def test_pins_catch_planted_mistake(tmp_path, monkeypatch, name):
 def test_unmutated_oracle_passes_suite():
     oracle._lib = None
     _pin_suite(oracle)
+
+
+# ------------------------------------------------- rotary + KV append (numpy)
+# Each case plants one mistake in a private copy of the source of
+# oracle.rope_append, executes it in a copy of the oracle module's namespace,
+# and checks that the rotary pins fail.
+
+ROPE_MUTATIONS = {
+    "rotation_sign": ("out[i] = vec[i] * c - vec[i + half] * s", "out[i] = vec[i] * c + vec[i + half] * s"),
+    "cos_sin_swapped": ("c, s = cos[pos, i], sin[pos, i]", "c, s = sin[pos, i], cos[pos, i]"),
+    "position_ignores_past": ("pos = past[b] + s", "pos = s"),
+    "k_from_v_slot": ("kc[b, h, pos] = rotate(row[(Hq + h) * d:(Hq + h + 1) * d], pos)",
+                      "kc[b, h, pos] = rotate(row[(Hq + Hkv + h) * d:(Hq + Hkv + h + 1) * d], pos)"),
+    "v_rotated": ("vc[b, h, pos] = row[(Hq + Hkv + h) * d:(Hq + Hkv + h + 1) * d]",
+                  "vc[b, h, pos] = rotate(row[(Hq + Hkv + h) * d:(Hq + Hkv + h + 1) * d], pos)"),
+    "adjacent_pairs": ("""            out[i] = vec[i] * c - vec[i + half] * s
+            out[i + half] = vec[i + half] * c + vec[i] * s""",
+                       """            out[2 * i] = vec[2 * i] * c - vec[2 * i + 1] * s
+            out[2 * i + 1] = vec[2 * i + 1] * c + vec[2 * i] * s"""),
+    "total_off_by_one": ("[p + S_new for p in past]", "[p + S_new - 1 for p in past]"),
+}
+
+
+def _rope_pin_suite(mod):
+    pins.test_rope_relative_position_property(mod)
+    pins.test_rope_append_positions_norms_and_untouched_rows(mod)
+    pins.test_rope_quarter_turn_closed_form(mod)
+
+
+@pytest.mark.parametrize("name", sorted(ROPE_MUTATIONS))
+def test_rope_pins_catch_planted_mistake(name):
+    import inspect
+    import textwrap
+    import types
+    old, new = ROPE_MUTATIONS[name]
+    src = textwrap.dedent(inspect.getsource(oracle.rope_append))
+    assert src.count(old) == 1, f"mutation anchor for {name} not unique"
+    namespace = dict(vars(oracle))
+    exec(compile(src.replace(old, new), f"<mutant {name}>", "exec"), namespace)
+    with pytest.raises(AssertionError):
+        _rope_pin_suite(types.SimpleNamespace(rope_append=namespace["rope_append"]))
+
+
+def test_unmutated_rope_oracle_passes_suite():
+    _rope_pin_suite(oracle)
