@@ -68,6 +68,7 @@ def bind(lib):
     lib.oracle_attn_rows_bias.argtypes = [_D, _D, _D, _D, i, i, i, i, i, i, i, i, d, i,
                                           _I64, ctypes.c_int64, _D, _D, i]
     lib.oracle_online_attn.argtypes = [_D, _D, _D, _D, _D, i, i, i, i, i, i, d, i, i, i]
+    lib.oracle_attn_bwd.argtypes = [_D, _D, _D, _D, _D, _D, _D, i, i, i, i, i, i, d, i, i]
     lib.oracle_split_partials.argtypes = [_D, _D, _D, i, i, i, i, i, i, d, i,
                                           _I32, i, _D, _D, _D]
     lib.oracle_split_combine.argtypes = [_D, _D, _D, ctypes.c_int64, i, i, _D, _D]
@@ -137,6 +138,29 @@ def attn_fwd(q, k, v, scale: float, causal: int = CAUSAL_NONE, nthreads: int | N
     if st != 0:
         raise ValueError(f"oracle_attn_fwd failed ({st})")
     return o, lse
+
+
+def attn_bwd(q, k, v, dout, scale: float, causal: int = CAUSAL_NONE, nthreads: int | None = None):
+    """Gradients (dq, dk, dv) of a loss whose gradient with respect to the
+    output o = attn_fwd(q, k, v, scale, causal) is ``dout`` ([B, Hq, Sq, d]).
+
+    The pages report the backward pass's speed but give no algorithm; this is
+    the chain rule through the five naive steps (sdpa_oracle.c,
+    oracle_attn_bwd), in fp64.  dk and dv of a KV head sum over the query heads
+    that share it.
+    """
+    q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Hq, Hkv, Sq, Sk, d = _dims(q, k, v)
+    if g.shape != q.shape:
+        raise ValueError("dout must have q's shape")
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    st = _load().oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dq), _ptr(dk), _ptr(dv),
+                                 B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal), _threads(nthreads))
+    if st != 0:
+        raise RuntimeError(f"oracle_attn_bwd failed ({st})")
+    return dq, dk, dv
 
 
 def attn_rows(q, k, v, scale: float, causal: int, rows, nthreads: int | None = None, bias=None):

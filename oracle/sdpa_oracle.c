@@ -27,6 +27,9 @@
  *    bias has two leading dimensions that broadcast over batch and heads
  *    (attn_bias_dim0 / attn_bias_dim1, 1 when absent).  oracle_attn_fwd_bias /
  *    oracle_attn_rows_bias.
+ *  - The backward pass (oracle_attn_bwd): the pages report its speed but give
+ *    no algorithm; the oracle is the chain rule through the five steps above
+ *    (see the comment at oracle_attn_bwd).
  *
  * Readings (where the pages are silent):
  *  - Bias: shape [bias_b, bias_h, Sq, Sk] with bias_b in {1, B} and bias_h in
@@ -69,17 +72,19 @@ static int key_visible(int causal, int i, int j, int Sq, int Sk) {
 }
 
 /*
- * The five naive steps for ONE query row (b, hq, i).  scores is scratch of Sk
- * doubles.  Writes o_row[d] and *lse_out.
+ * Steps 1-4 of the naive definition for ONE query row (b, hq, i): scores
+ * (scratch of Sk doubles) receives the softmax probabilities of the row.
+ * Returns 1 for a fully masked row (all probabilities 0), else 0 with the
+ * row max *mx_out and denominator *sum_out.  *hk_out is the row's KV head.
  */
-static void attn_one_row(const attn_args *a, int b, int hq, int i,
-                         double *scores, double *o_row, double *lse_out) {
+static int attn_probs_row(const attn_args *a, int b, int hq, int i, double *scores,
+                          double *mx_out, double *sum_out, int *hk_out) {
     const int d = a->d, Sk = a->Sk;
     const int group = a->Hq / a->Hkv;
     const int hk = hq / group;
     const double *qrow = a->q + (((size_t)b * a->Hq + hq) * a->Sq + i) * d;
     const double *kbase = a->k + ((size_t)b * a->Hkv + hk) * (size_t)Sk * d;
-    const double *vbase = a->v + ((size_t)b * a->Hkv + hk) * (size_t)Sk * d;
+    *hk_out = hk;
 
     /* step 1: scores = q . k^T */
     for (int j = 0; j < Sk; ++j) {
@@ -103,9 +108,8 @@ static void attn_one_row(const attn_args *a, int b, int hq, int i,
     for (int j = 0; j < Sk; ++j)
         if (scores[j] > mx) mx = scores[j];
     if (mx == -INFINITY) {
-        for (int c = 0; c < d; ++c) o_row[c] = 0.0;
-        *lse_out = -INFINITY;
-        return;
+        for (int j = 0; j < Sk; ++j) scores[j] = 0.0;
+        return 1;
     }
     double sum = 0.0;
     for (int j = 0; j < Sk; ++j) {
@@ -113,6 +117,26 @@ static void attn_one_row(const attn_args *a, int b, int hq, int i,
         sum += scores[j];
     }
     for (int j = 0; j < Sk; ++j) scores[j] /= sum;
+    *mx_out = mx;
+    *sum_out = sum;
+    return 0;
+}
+
+/*
+ * The five naive steps for ONE query row (b, hq, i).  scores is scratch of Sk
+ * doubles.  Writes o_row[d] and *lse_out.
+ */
+static void attn_one_row(const attn_args *a, int b, int hq, int i,
+                         double *scores, double *o_row, double *lse_out) {
+    const int d = a->d, Sk = a->Sk;
+    double mx = 0.0, sum = 0.0;
+    int hk = 0;
+    if (attn_probs_row(a, b, hq, i, scores, &mx, &sum, &hk)) {
+        for (int c = 0; c < d; ++c) o_row[c] = 0.0;
+        *lse_out = -INFINITY;
+        return;
+    }
+    const double *vbase = a->v + ((size_t)b * a->Hkv + hk) * (size_t)Sk * d;
     /* step 5: out = attn . v */
     for (int c = 0; c < d; ++c) o_row[c] = 0.0;
     for (int j = 0; j < Sk; ++j) {
@@ -250,6 +274,121 @@ int oracle_attn_rows_bias(const double *q, const double *k, const double *v, con
         if (rows[r] < 0 || rows[r] >= total) return -1;
     attn_args a = {q, k, v, NULL, NULL, B, Hq, Hkv, Sq, Sk, d, scale, causal, bias, bias_b, bias_h};
     return run_rows(&a, rows, n, o_rows, lse_rows, nthreads);
+}
+
+/* ------------------------------------------------------- backward pass */
+
+/*
+ * Gradients of a scalar loss L through the five steps, given dout = dL/do
+ * ([B, Hq, Sq, d]).  The pages give no backward algorithm; this is the chain
+ * rule through the plain definition, one query row at a time (P = the row's
+ * softmax probabilities from steps 1-4, x = the scaled scores):
+ *   dP_ij = dout_i . v_j                      (step 5: o_i = sum_j P_ij v_j)
+ *   dx_ij = P_ij (dP_ij - sum_k P_ik dP_ik)   (step 4: softmax Jacobian; masked
+ *                                              keys have P_ij = 0, so dx_ij = 0)
+ *   dq_i  = scale sum_j dx_ij k_j,  dk_j += scale dx_ij q_i   (steps 1-2)
+ *   dv_j += P_ij dout_i                                        (step 5)
+ * With GQA, dk and dv of a KV head sum over the query heads that read it.
+ * One job per (batch, KV head) owns its dk/dv rows, so jobs never share a sum.
+ */
+typedef struct {
+    const attn_args *a;
+    const double *dout;
+    double *dq, *dk, *dv;
+    int64_t begin, end; /* flattened (b * Hkv + hk) */
+    int status;
+} bwd_job;
+
+static void *bwd_worker(void *p) {
+    bwd_job *job = (bwd_job *)p;
+    const attn_args *a = job->a;
+    const int d = a->d, Sk = a->Sk, Sq = a->Sq, group = a->Hq / a->Hkv;
+    double *probs = (double *)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+    double *dprob = (double *)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+    if (!probs || !dprob) { free(probs); free(dprob); job->status = -2; return NULL; }
+    for (int64_t bk = job->begin; bk < job->end; ++bk) {
+        const int b = (int)(bk / a->Hkv), hk = (int)(bk % a->Hkv);
+        const double *kbase = a->k + ((size_t)b * a->Hkv + hk) * (size_t)Sk * d;
+        const double *vbase = a->v + ((size_t)b * a->Hkv + hk) * (size_t)Sk * d;
+        double *dkbase = job->dk + ((size_t)b * a->Hkv + hk) * (size_t)Sk * d;
+        double *dvbase = job->dv + ((size_t)b * a->Hkv + hk) * (size_t)Sk * d;
+        for (int hq = hk * group; hq < (hk + 1) * group; ++hq) {
+            for (int i = 0; i < Sq; ++i) {
+                const size_t row = ((size_t)b * a->Hq + hq) * Sq + i;
+                const double *qrow = a->q + row * d;
+                const double *grow = job->dout + row * d;
+                double *dqrow = job->dq + row * d;
+                for (int c = 0; c < d; ++c) dqrow[c] = 0.0;
+                double mx = 0.0, sum = 0.0;
+                int hk_row = 0;
+                if (attn_probs_row(a, b, hq, i, probs, &mx, &sum, &hk_row)) continue; /* no visible key */
+                /* dP_ij = dout_i . v_j and D_i = sum_j P_ij dP_ij */
+                double D = 0.0;
+                for (int j = 0; j < Sk; ++j) {
+                    double s = 0.0;
+                    for (int c = 0; c < d; ++c) s += grow[c] * vbase[(size_t)j * d + c];
+                    dprob[j] = s;
+                    D += probs[j] * s;
+                }
+                for (int j = 0; j < Sk; ++j) {
+                    const double pj = probs[j];
+                    if (pj == 0.0) continue;
+                    const double dx = pj * (dprob[j] - D);
+                    const double *krow = kbase + (size_t)j * d;
+                    double *dkrow = dkbase + (size_t)j * d;
+                    double *dvrow = dvbase + (size_t)j * d;
+                    for (int c = 0; c < d; ++c) {
+                        dqrow[c] += a->scale * dx * krow[c];
+                        dkrow[c] += a->scale * dx * qrow[c];
+                        dvrow[c] += pj * grow[c];
+                    }
+                }
+            }
+        }
+    }
+    free(probs);
+    free(dprob);
+    job->status = 0;
+    return NULL;
+}
+
+/* dq [B,Hq,Sq,d], dk and dv [B,Hkv,Sk,d] for dout [B,Hq,Sq,d] (no bias). */
+int oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dout,
+                    double *dq, double *dk, double *dv,
+                    int B, int Hq, int Hkv, int Sq, int Sk, int d, double scale, int causal,
+                    int nthreads) {
+    if (check_shape(B, Hq, Hkv, Sq, Sk, d, causal)) return -1;
+    memset(dk, 0, sizeof(double) * (size_t)B * Hkv * Sk * d);
+    memset(dv, 0, sizeof(double) * (size_t)B * Hkv * Sk * d);
+    memset(dq, 0, sizeof(double) * (size_t)B * Hq * Sq * d);
+    const int64_t njobs = (int64_t)B * Hkv;
+    if (njobs == 0) return 0;
+    attn_args a = {q, k, v, NULL, NULL, B, Hq, Hkv, Sq, Sk, d, scale, causal, NULL, 1, 1};
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > njobs) nthreads = (int)njobs;
+    bwd_job *jobs = (bwd_job *)calloc((size_t)nthreads, sizeof(bwd_job));
+    pthread_t *tids = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    char *joinable = (char *)calloc((size_t)nthreads, 1);
+    if (!jobs || !tids || !joinable) { free(jobs); free(tids); free(joinable); return -2; }
+    const int64_t per = (njobs + nthreads - 1) / nthreads;
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t].a = &a; jobs[t].dout = dout; jobs[t].dq = dq; jobs[t].dk = dk; jobs[t].dv = dv;
+        jobs[t].begin = (int64_t)t * per;
+        jobs[t].end = jobs[t].begin + per < njobs ? jobs[t].begin + per : njobs;
+        jobs[t].status = -3;
+        if (jobs[t].begin >= jobs[t].end) { jobs[t].status = 0; continue; }
+        if (pthread_create(&tids[t], NULL, bwd_worker, &jobs[t]) == 0)
+            joinable[t] = 1;
+        else
+            bwd_worker(&jobs[t]);
+    }
+    int status = 0;
+    for (int t = 0; t < nthreads; ++t) {
+        if (joinable[t]) pthread_join(tids[t], NULL);
+        if (jobs[t].status != 0) status = jobs[t].status;
+    }
+    free(jobs); free(tids); free(joinable);
+    return status;
 }
 
 /* ------------------------------------------------- FA2 online recurrence */

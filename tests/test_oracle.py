@@ -484,3 +484,87 @@ def test_rope_quarter_turn_closed_form(oracle_mod):
                                          np.zeros((1, 1, cap, d)), 1, 1)
     assert np.array_equal(q[0, 0, 0], np.array([-3.0, -4.0, 1.0, 2.0]))
     assert np.array_equal(kc[0, 0, 1], np.array([-7.0, -8.0, 5.0, 6.0]))
+
+
+# ------------------------------------------------------------ backward pass
+# (the pages give no backward algorithm; the oracle is the chain rule through
+# the five naive steps, pinned here by finite differences of the forward
+# oracle and by properties of the softmax Jacobian)
+
+def _bwd_inputs(B, Hq, Hkv, Sq, Sk, d, seed):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((B, Hq, Sq, d)), rng.standard_normal((B, Hkv, Sk, d)),
+            rng.standard_normal((B, Hkv, Sk, d)), rng.standard_normal((B, Hq, Sq, d)))
+
+
+@pytest.mark.parametrize("causal", [0, 1, 2])
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,d", [(1, 1, 1, 3, 4, 3), (2, 2, 1, 4, 3, 2), (1, 2, 2, 5, 5, 4)])
+def test_bwd_matches_finite_differences(oracle_mod, B, Hq, Hkv, Sq, Sk, d, causal):
+    """Every entry of dq, dk, dv equals the central difference of
+    L = sum(o * dout) through the forward oracle (h = 1e-5: truncation and
+    rounding errors both below 1e-9)."""
+    q, k, v, g = _bwd_inputs(B, Hq, Hkv, Sq, Sk, d, 100 + causal)
+    scale = 0.6
+    dq, dk, dv = oracle_mod.attn_bwd(q, k, v, g, scale, causal)
+    loss = lambda qq, kk, vv: float((oracle_mod.attn_fwd(qq, kk, vv, scale, causal)[0] * g).sum())
+    h = 1e-5
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        base = [q, k, v]
+        for idx in np.ndindex(*base[which].shape):
+            plus = [x.copy() for x in base]
+            minus = [x.copy() for x in base]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            fd = (loss(*plus) - loss(*minus)) / (2 * h)
+            assert abs(fd - grad[idx]) < 1e-8, (which, idx, fd, grad[idx])
+
+
+def test_bwd_single_key_closed_form(oracle_mod):
+    """With one key every output row is v_0: dv_0 sums dout over all rows of
+    every query head of the group, and q and k get no gradient."""
+    q, k, v, g = _bwd_inputs(2, 4, 2, 5, 1, 3, 110)
+    dq, dk, dv = oracle_mod.attn_bwd(q, k, v, g, 0.5, 0)
+    assert np.array_equal(dq, np.zeros_like(dq)) and np.array_equal(dk, np.zeros_like(dk))
+    for b in range(2):
+        for hk in range(2):
+            expect = g[b, 2 * hk:2 * hk + 2].sum(axis=(0, 1))
+            assert np.allclose(dv[b, hk, 0], expect, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [0, 1, 2])
+def test_bwd_key_gradients_sum_to_zero_and_key_shift_leaves_dq(oracle_mod, causal):
+    """Each row of the softmax Jacobian sums to zero, so sum_j dk_j = 0; and
+    adding one vector to every key shifts a row's scores by a constant, so o
+    and dq do not change."""
+    q, k, v, g = _bwd_inputs(2, 2, 1, 6, 6, 4, 120 + causal)
+    dq, dk, dv = oracle_mod.attn_bwd(q, k, v, g, 0.8, causal)
+    assert np.abs(dk.sum(axis=2)).max() < 1e-12
+    shift = np.random.default_rng(5).standard_normal(4)
+    dq2, _, _ = oracle_mod.attn_bwd(q, k + shift, v, g, 0.8, causal)
+    assert np.abs(dq2 - dq).max() < 1e-10
+
+
+@pytest.mark.parametrize("causal", [0, 1, 2])
+def test_bwd_gqa_equals_explicit_expansion(oracle_mod, causal):
+    """dk, dv of a shared KV head = the sum over its query heads of the
+    gradients with K/V repeated per query head."""
+    q, k, v, g = _bwd_inputs(1, 4, 2, 5, 6, 3, 130 + causal)
+    dq, dk, dv = oracle_mod.attn_bwd(q, k, v, g, 0.7, causal)
+    ke, ve = np.repeat(k, 2, axis=1), np.repeat(v, 2, axis=1)
+    dqe, dke, dve = oracle_mod.attn_bwd(q, ke, ve, g, 0.7, causal)
+    assert np.allclose(dq, dqe, atol=1e-12)
+    assert np.allclose(dk, dke.reshape(1, 2, 2, 6, 3).sum(axis=2), atol=1e-12)
+    assert np.allclose(dv, dve.reshape(1, 2, 2, 6, 3).sum(axis=2), atol=1e-12)
+
+
+def test_bwd_masked_rows_and_unseen_keys_get_no_gradient(oracle_mod):
+    """Bottom-right with Sq > Sk: the first Sq - Sk rows see no key, so their
+    dq is 0.  Top-left with Sk > Sq: keys j >= Sq are seen by no row, so their
+    dk and dv are 0."""
+    q, k, v, g = _bwd_inputs(1, 1, 1, 6, 3, 4, 140)
+    dq, dk, dv = oracle_mod.attn_bwd(q, k, v, g, 0.5, 2)
+    assert np.array_equal(dq[0, 0, :3], np.zeros((3, 4)))
+    assert np.abs(dq[0, 0, 3:]).max() > 0
+    q, k, v, g = _bwd_inputs(1, 1, 1, 3, 6, 4, 141)
+    dq, dk, dv = oracle_mod.attn_bwd(q, k, v, g, 0.5, 1)
+    assert np.array_equal(dk[0, 0, 3:], np.zeros((3, 4))) and np.array_equal(dv[0, 0, 3:], np.zeros((3, 4)))

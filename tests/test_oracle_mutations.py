@@ -36,6 +36,11 @@ MUTATIONS = {
     "bias_broadcast_swapped": ("const int bb = a->bias_b == 1 ? 0 : b, bh = a->bias_h == 1 ? 0 : hq;",
                                "const int bb = a->bias_h == 1 ? 0 : b, bh = a->bias_b == 1 ? 0 : hq;"),
     "bias_row_index": ("* a->Sq + i) * (size_t)Sk;", "* a->Sq + (a->Sq - 1 - i)) * (size_t)Sk;"),
+    "bwd_no_jacobian_mean": ("const double dx = pj * (dprob[j] - D);", "const double dx = pj * dprob[j];"),
+    "bwd_dk_unscaled": ("dkrow[c] += a->scale * dx * qrow[c];", "dkrow[c] += dx * qrow[c];"),
+    "bwd_dv_from_dx": ("dvrow[c] += pj * grow[c];", "dvrow[c] += dx * grow[c];"),
+    "bwd_dq_from_v": ("dqrow[c] += a->scale * dx * krow[c];",
+                      "dqrow[c] += a->scale * dx * vbase[(size_t)j * d + c];"),
 }
 
 
@@ -55,6 +60,8 @@ def _pin_suite(mod):
     for dims in ((1, 1), (2, 1), (1, 4), (2, 4)):
         pins.test_bias_brute_force_every_broadcast(mod, dims, 1)
     pins.test_bias_of_log_weights_with_zero_query_is_weighted_mean(mod)
+    pins.test_bwd_matches_finite_differences(mod, 2, 2, 1, 4, 3, 2, 2)
+    pins.test_bwd_single_key_closed_form(mod)
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
