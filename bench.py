@@ -335,6 +335,28 @@ class GpuDecodeVarlen(GpuDecode):
         return kv + 2 * w.B * w.Hq * w.Sq * w.d * 2 + w.B * w.Hq * w.Sq * 4
 
 
+class GpuBackward(GpuPrefill):
+    """attn_bwd on a prefill workload, with the forward's o and lse and a
+    seeded dO resident on the device."""
+
+    def __init__(self, w, rank: int):
+        import scaled_dot_product_fa2_b200 as sdpa
+        super().__init__(w, rank)
+        sdpa.attn_fwd(self.q, self.k, self.v, causal=w.causal, scale=w.scale, out=self.o, lse=self.lse)
+        g = torch.Generator().manual_seed(w.seed + 4242 + 7919 * rank)
+        self.dout = torch.randn(self.q.shape, generator=g).bfloat16().cuda()
+        self.dq = torch.empty_like(self.q)
+        self.dk = torch.empty_like(self.k)
+        self.dv = torch.empty_like(self.v)
+        self.ws = torch.empty(max(16, sdpa.ops._lib.get().attn_bwd_workspace_size(w.B, w.Hq, w.Sq)),
+                              dtype=torch.uint8, device="cuda")
+
+    def run(self):
+        import scaled_dot_product_fa2_b200 as sdpa
+        sdpa.attn_bwd(self.q, self.k, self.v, self.o, self.lse, self.dout, causal=self.w.causal, scale=self.w.scale,
+                      dq=self.dq, dk=self.dk, dv=self.dv, workspace=self.ws)
+
+
 class GpuRopeAppend:
     """The step before a decode: split the packed QKV, rotate q and k, append
     k and v to the cache (one launch of the rotary/append kernel)."""
@@ -576,6 +598,16 @@ def measure_breakdown(flush, peak_tf, hbm_gbs, rank, reps: int = 10):
         gbs = s.valid_bytes() / ms / 1e6
         out[w.name + "_varlen"] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4),
                                    "lengths": s.lens, "launches_per_call": 2}
+        del s
+    # backward pass at seq 4096 (B=4, H=16, d=128): the forward's o, lse are
+    # computed once outside the timing; FLOPs = 2.5 x the forward's (the five
+    # matmuls S = QK^T, dP = dO V^T, dV, dK, dQ), halved for causal
+    for name in ("prefill_noncausal_s4096", "prefill_causal_s4096"):
+        s = GpuBackward(inputs.BY_NAME[name], rank)
+        ms = statistics.median(timed_calls([s.run], flush, reps, 3)[0])
+        tf = 2.5 * s.w.flops() / ms / 1e9
+        out["bwd_" + name.replace("prefill_", "")] = {"ms": round(ms, 4), "tflops": round(tf, 1),
+                                                       "frac": round(tf / peak_tf, 4), "launches_per_call": 3}
         del s
     # rotary/append over a 4096-token prompt: 805 MB moved per call (> L2), no flush needed
     s = GpuRopeAppend(inputs.ROPE_PROMPT, rank)

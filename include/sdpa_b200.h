@@ -265,6 +265,33 @@ attn_status_t attn_decode_splitkv_static(const void* q, const void* k_cache, con
                                          int causal, int num_splits, void* stream);
 
 /*
+ * Backward pass of attn_fwd: gradients dq, dk, dv of a loss L given
+ * dout = dL/do.  "FlashAttention-2" notes report the backward pass's speed
+ * but give no algorithm; this library's kernels recompute the probabilities
+ * P = exp(scale q.k - lse) tile by tile from the forward's lse (nothing of
+ * size Sq x Sk is stored) and apply the chain rule through the forward:
+ *   dP = dout v^T,  D_i = dout_i . o_i,  dS = P (dP - D),
+ *   dq = scale dS k,  dk = scale dS^T q,  dv = P^T dout,
+ * with dk and dv of a KV head summed over the query heads that share it (GQA).
+ *
+ *   q, o, dout, dq   [B, Hq, Sq, d] bf16 (BHSD), device
+ *   k, v, dk, dv     [B, Hkv, Sk, d] bf16, device
+ *   lse              [B, Hq, Sq] fp32: the forward's lse (natural log) for the
+ *                    same q, k, v, scale and causal mode; o is its output.
+ *   workspace        attn_bwd_workspace_size(B, Hq, Sq) bytes, device,
+ *                    16-byte aligned, caller-owned; nothing in it needs to be
+ *                    initialised.
+ * scale and causal as in attn_fwd (causal 0, 1 or 2).  Every output is fully
+ * written: rows that saw no key get dq = 0; keys no row sees get dk = dv = 0;
+ * Sq == 0 gives dk = dv = 0, Sk == 0 gives dq = 0.  Errors as attn_fwd, plus
+ * ATTN_ERR_WORKSPACE.  Three kernels on `stream`, asynchronous.
+ */
+size_t attn_bwd_workspace_size(int B, int Hq, int Sq);
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                       float scale, int causal, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * The step before a decode: split a packed QKV projection, rotate q and k by
  * the rotary embedding, append k and v to the KV cache -- one streaming kernel.
  * This is the fused "split packed QKV with rotary embedding and copy KV" step

@@ -1,0 +1,544 @@
+// backward.cuh -- gradients of the fused attention forward for sm_100a.
+//
+// For a loss L with dO = dL/dO, the forward's P = softmax(scale Q K^T + mask)
+// and O = P V give (one query row i, key j):
+//   dP_ij = dO_i . V_j,   dS_ij = P_ij (dP_ij - D_i),   D_i = sum_j P_ij dP_ij
+//   dQ_i = scale sum_j dS_ij K_j,   dK_j = scale sum_i dS_ij Q_i,   dV_j = sum_i P_ij dO_i
+// and D_i also equals dO_i . O_i, since O_i = sum_j P_ij V_j.  The pages
+// report the FlashAttention-2 backward's speed ("FlashAttention-2" notes) but
+// give no algorithm; this file is this library's own design: P is recomputed
+// from the forward's LSE (P_ij = exp(scale q_i.k_j - LSE_i)), so nothing of
+// size Sq x Sk is ever stored.
+//
+// Three kernels:
+//   bwd_prep_kernel   D_i = dO_i . O_i and LSE_i in log2 units, into the
+//                     caller's workspace (rows padded to whole 128-row tiles:
+//                     padding has D = 0 and LSE = +inf, i.e. P = 0).
+//   bwd_dkdv_kernel   one CTA per 128-key tile of a (batch, KV head): K and V
+//                     stay in shared memory while the query tiles of every
+//                     query head of the group stream through a 2-stage ring.
+//                     Per query tile: S^T = K Q^T and dP^T = V dO^T (tcgen05,
+//                     into TMEM), P^T and dS^T by the four compute warps (one
+//                     thread per key row, written back to TMEM as bf16 over
+//                     the first half of S^T and dP^T), then dV += P^T dO and
+//                     dK += dS^T Q with P^T, dS^T read from TMEM.
+//   bwd_dq_kernel     one CTA per 128-row query tile: Q and dO stay in shared
+//                     memory while the key tiles stream; S = Q K^T and
+//                     dP = dO V^T, dS by the compute warps, dQ += dS K.
+// Fully masked key tiles are skipped (causal).  TMEM holds every accumulator
+// (dK and dV for the whole query loop, dQ for the whole key loop).  Every
+// wait is bounded; a timeout sets the device error word and the kernel exits.
+#pragma once
+#include "prefill.cuh"
+
+namespace sdpa {
+
+struct BwdParams {
+  // 4-D maps (d, S, H, B) over q, k, v, dO (BHSD); box {64, 128, 1, 1}, 128-byte swizzle.
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  CUtensorMap tm_do;
+  const uint16_t* o;    // forward output, bf16 [B, Hq, Sq, d]
+  const uint16_t* dout;  // dO, bf16 [B, Hq, Sq, d]
+  const float* lse;     // forward LSE (natural log) [B, Hq, Sq]
+  float* l2;            // workspace [B*Hq][Sq_pad]: LSE * log2(e), +inf where P = 0
+  float* dvec;          // workspace [B*Hq][Sq_pad]: D = rowsum(dO * O)
+  uint16_t* dq;         // bf16 [B, Hq, Sq, d]
+  uint16_t* dk;         // bf16 [B, Hkv, Sk, d]
+  uint16_t* dv;         // bf16 [B, Hkv, Sk, d]
+  int B, Hq, Hkv, Sq, Sk, Sq_pad, group;
+  int causal;    // 0 none, 1 top-left, 2 bottom-right
+  int coff;      // key j visible to row i iff j <= i + coff (causal)
+  int n_qt, n_kt;  // query / key tiles of 128
+  float scale;       // softmax scale
+  float scale_log2;  // scale * log2(e)
+};
+
+constexpr int kBwdThreads = 192;  // warps 0-3 compute, 4 MMA issuer (+ TMEM owner), 5 TMA producer
+constexpr int kBwdMmaWarp = 4;
+constexpr int kBwdLoadWarp = 5;
+constexpr int kBwdStages = 2;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// 1-D bulk copy global -> shared (no tensor map), completion counted on `bar`.
+// Both addresses 16-byte aligned, `bytes` a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t smem_dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit TMEM columns from registers.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kTileBytes = 128 * D * 2;   // one 128-row bf16 tile
+  static constexpr int kBlocks = D / 64;            // 64-column swizzle blocks per tile
+  static constexpr int kBlockBytes = 128 * 128;     // 16 KB per swizzle block
+  static constexpr int kVecBytes = 128 * 4;         // 128 fp32 (L2 or D of one query tile)
+  // smem: two resident tiles, then per stage two streamed tiles and two vectors
+  static constexpr int kStageBytes = 2 * kTileBytes + 2 * kVecBytes;
+  // res_full, st_full[2], st_empty[2], s_full, p_full, done
+  static constexpr int kNumBars = 1 + 2 * kBwdStages + 3;
+  static constexpr int kSmemBytes = 2 * kTileBytes + kBwdStages * kStageBytes + kNumBars * 8 + 16 + 1024;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
+  static constexpr uint32_t kTmemCols = 512;
+  // Each CTA takes all 512 TMEM columns, and tcgen05.alloc waits without a
+  // bound for columns another CTA holds: launch with more than half of the
+  // SM's 228 KB of shared memory, so that no two CTAs share an SM.
+  static constexpr int kSmemLaunch = kSmemBytes > 116 * 1024 ? kSmemBytes : 116 * 1024;
+};
+
+// -------------------------------------------------------------- prep kernel
+// One warp per padded row: D = dO . O (fp32) and LSE * log2(e).  A row that
+// saw no key has LSE = -inf and a padding row has none: both get +inf, so
+// that exp2(x - l2) = 0 for them.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __grid_constant__ BwdParams p) {
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= static_cast<int64_t>(p.B) * p.Hq * p.Sq_pad) return;
+  const int i = static_cast<int>(w % p.Sq_pad);
+  const int64_t bh = w / p.Sq_pad;
+  float dsum = 0.f, l2 = INFINITY;
+  if (i < p.Sq) {
+    const int64_t row = (bh * p.Sq + i) * D;
+    constexpr int kPer = D / 32;  // bf16 elements per lane: 4 (d=128) or 2 (d=64)
+    const uint16_t* orow = p.o + row + lane * kPer;
+    const uint16_t* grow = p.dout + row + lane * kPer;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) dsum += bf16_bits_to_float(__ldg(orow + e)) * bf16_bits_to_float(__ldg(grow + e));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
+    const float lse = __ldg(p.lse + bh * p.Sq + i);
+    l2 = (lse == -INFINITY) ? INFINITY : lse * kLog2e;
+  }
+  if (lane == 0) {
+    p.dvec[w] = dsum;
+    p.l2[w] = l2;
+  }
+}
+
+// ------------------------------------------------------------ dK, dV kernel
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
+  using Cfg = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // K | V | stage 0: Q, dO, L2, D | stage 1: ... | barriers
+  const uint32_t sK = smem_u32(smem);
+  const uint32_t sV = sK + Cfg::kTileBytes;
+  auto sQ = [&](int st) { return sK + 2 * Cfg::kTileBytes + st * Cfg::kStageBytes; };
+  auto sDO = [&](int st) { return sQ(st) + Cfg::kTileBytes; };
+  const float* vec_base = reinterpret_cast<const float*>(smem + 2 * Cfg::kTileBytes + 2 * Cfg::kTileBytes);
+  auto l2_at = [&](int st) { return vec_base + st * (Cfg::kStageBytes / 4); };
+  auto dd_at = [&](int st) { return vec_base + st * (Cfg::kStageBytes / 4) + 128; };
+  const uint32_t bar0 = sK + 2 * Cfg::kTileBytes + kBwdStages * Cfg::kStageBytes;
+  const uint32_t res_full = bar0;
+  auto st_full = [&](int st) { return bar0 + 8u * (1 + st); };
+  auto st_empty = [&](int st) { return bar0 + 8u * (1 + kBwdStages + st); };
+  const uint32_t s_full = bar0 + 8u * (1 + 2 * kBwdStages);
+  const uint32_t p_full = s_full + 8u;
+  const uint32_t done = p_full + 8u;
+  uint8_t* bar_ptr = smem + 2 * Cfg::kTileBytes + kBwdStages * Cfg::kStageBytes;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * Cfg::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int kt = static_cast<int>(blockIdx.x % p.n_kt);
+  const int bkv = static_cast<int>(blockIdx.x / p.n_kt);
+  const int b = bkv / p.Hkv;
+  const int hkv = bkv - b * p.Hkv;
+  const int k0 = kt * 128;
+  // query tiles that see any key of this tile: rows i >= k0 - coff (causal)
+  const int qt0 = p.causal ? max(0, (k0 - p.coff) / 128) : 0;
+  const int per_head = max(0, p.n_qt - qt0);
+  const int n_it = per_head * p.group;
+
+  if (threadIdx.x == 0) {
+    mbar_init(res_full, 1);
+    for (int st = 0; st < kBwdStages; ++st) {
+      mbar_init(st_full(st), 1);
+      mbar_init(st_empty(st), 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);  // one arrive per compute warp
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM columns: S^T [0,128) | dP^T [128,256) | dV [256,256+D) | dK [256+D,256+2D)
+  constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+
+  if (warp == kBwdLoadWarp) {
+    if (lane == 0 && n_it > 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_do);
+      mbar_arrive_expect_tx(res_full, 2 * Cfg::kTileBytes);
+      for (int blk = 0; blk < Cfg::kBlocks; ++blk) {
+        tma_load_4d(sK + blk * Cfg::kBlockBytes, &p.tm_k, blk * 64, k0, hkv, b, res_full);
+        tma_load_4d(sV + blk * Cfg::kBlockBytes, &p.tm_v, blk * 64, k0, hkv, b, res_full);
+      }
+      int it = 0;
+      for (; it < n_it; ++it) {
+        const int st = it % kBwdStages;
+        if (!mbar_wait(st_empty(st), ((it / kBwdStages) & 1) ^ 1, abort_flag)) break;
+        const int hq = hkv * p.group + it / per_head;
+        const int qt = qt0 + it % per_head;
+        mbar_arrive_expect_tx(st_full(st), 2 * Cfg::kTileBytes + 2 * Cfg::kVecBytes);
+        for (int blk = 0; blk < Cfg::kBlocks; ++blk) {
+          tma_load_4d(sQ(st) + blk * Cfg::kBlockBytes, &p.tm_q, blk * 64, qt * 128, hq, b, st_full(st));
+          tma_load_4d(sDO(st) + blk * Cfg::kBlockBytes, &p.tm_do, blk * 64, qt * 128, hq, b, st_full(st));
+        }
+        const int64_t vec = (static_cast<int64_t>(b) * p.Hq + hq) * p.Sq_pad + qt * 128;
+        bulk_load(smem_u32(l2_at(st)), p.l2 + vec, Cfg::kVecBytes, st_full(st));
+        bulk_load(smem_u32(dd_at(st)), p.dvec + vec, Cfg::kVecBytes, st_full(st));
+      }
+      // copies in flight must land before the CTA may exit
+      mbar_wait_drain(res_full, 0);
+      for (int i = max(0, it - kBwdStages); i < it; ++i) mbar_wait_drain(st_full(i % kBwdStages), (i / kBwdStages) & 1);
+    }
+    __syncwarp();
+  } else if (warp == kBwdMmaWarp) {
+    if (lane == 0 && n_it > 0) {
+      const uint64_t hi = static_cast<uint64_t>(sdesc_hi(1024)) << 32;
+      const uint64_t dk_k = hi | sdesc_lo(sK, 16);  // K, K-major (A of S^T)
+      const uint64_t dv_k = hi | sdesc_lo(sV, 16);  // V, K-major (A of dP^T)
+      bool ok = mbar_wait(res_full, 0, abort_flag);
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int st = it % kBwdStages;
+        if (!mbar_wait(st_full(st), (it / kBwdStages) & 1, abort_flag)) break;
+        tc_fence_after();
+        // S^T = K Q^T, dP^T = V dO^T (M = 128 keys, N = 128 queries, K = D).
+        // They overwrite P^T, dS^T of the previous tile only after the MMAs
+        // reading them: one thread issues all MMAs, in order.
+        issue_qk<D>(tmem + kColS, dk_k, hi | sdesc_lo(sQ(st), 16));
+        issue_qk<D>(tmem + kColDP, dv_k, hi | sdesc_lo(sDO(st), 16));
+        mma_commit(s_full);
+        if (!mbar_wait(p_full, it & 1, abort_flag)) break;
+        tc_fence_after();
+        // dV += P^T dO, dK += dS^T Q (M = 128 keys, N = D, K = 128 queries;
+        // A from TMEM, B = the query-side tile, MN-major).
+        const uint64_t ddo_mn = hi | sdesc_lo(sDO(st), Cfg::kBlockBytes);
+        const uint64_t dq_mn = hi | sdesc_lo(sQ(st), Cfg::kBlockBytes);
+        issue_pv<D, 0>(tmem + kColDV, tmem + kColS, ddo_mn, it > 0);
+        issue_pv<D, 1>(tmem + kColDV, tmem + kColS, ddo_mn, true);
+        issue_pv<D, 0>(tmem + kColDK, tmem + kColDP, dq_mn, it > 0);
+        issue_pv<D, 1>(tmem + kColDK, tmem + kColDP, dq_mn, true);
+        mma_commit(st_empty(st));
+      }
+      mma_commit(done);
+      mbar_wait_drain(done, 0);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------ compute: one key row per thread
+    const int r = warp * 32 + lane;
+    const int j = k0 + r;
+    const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+    const float c = p.scale_log2;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int st = it % kBwdStages;
+      const int qt = qt0 + it % per_head;
+      // query columns c < cmin do not see key j (causal); keys past Sk see nothing
+      const int cmin = (j >= p.Sk) ? INT_MAX : (p.causal ? j - p.coff - qt * 128 : INT_MIN);
+      // S^T/dP^T ready; the stage's L2/D vectors landed (the wait on the
+      // stage's own barrier makes the bulk copy's writes visible here)
+      // (warp-uniform: the tcgen05.ld/st below are collective over the warp)
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag) &&
+                                       mbar_wait(st_full(st), (it / kBwdStages) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const float* l2v = l2_at(st);
+      const float* ddv = dd_at(st);
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t sv[32], dp[32];
+        tmem_ld32(tmem + lane_bits + kColS + ch * 32, sv);
+        tmem_ld32(tmem + lane_bits + kColDP + ch * 32, dp);
+        tmem_wait_ld();
+        uint32_t pk[16], dk16[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 lv = *reinterpret_cast<const float4*>(l2v + ch * 32 + e);
+          const float4 dv4 = *reinterpret_cast<const float4*>(ddv + ch * 32 + e);
+          const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
+          const float dq4[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+          float pr[4], ds[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int col = ch * 32 + e + u;
+            const float x = fmaf(__uint_as_float(sv[e + u]), c, -lq[u]);
+            pr[u] = (col >= cmin) ? ex2_approx(x) : 0.f;
+            ds[u] = pr[u] * (__uint_as_float(dp[e + u]) - dq4[u]);
+          }
+          pk[e / 2] = pack_bf16x2(pr[0], pr[1]);
+          pk[e / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
+          dk16[e / 2] = pack_bf16x2(ds[0], ds[1]);
+          dk16[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+        }
+        // chunk ch of S^T / dP^T is in registers; its bf16 result goes to
+        // columns already read (16 ch .. 16 ch + 15)
+        tmem_st16(tmem + lane_bits + kColS + ch * 16, pk);
+        tmem_st16(tmem + lane_bits + kColDP + ch * 16, dk16);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    // ---- epilogue: dK = scale * acc, dV = acc -> bf16 rows.  The TMEM loads
+    // are collective: the whole warp runs them (warp-uniform `have`); only
+    // the stores depend on the lane's row.
+    const bool have = __all_sync(0xffffffffu, ok && n_it > 0 && mbar_wait(done, 0, abort_flag));
+    if (have) tc_fence_after();
+    {
+      const int64_t row = ((static_cast<int64_t>(b) * p.Hkv + hkv) * p.Sk + j) * D;
+#pragma unroll 1
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t a[32], g[32];
+        if (have) {
+          tmem_ld32(tmem + lane_bits + kColDV + q * 32, a);
+          tmem_ld32(tmem + lane_bits + kColDK + q * 32, g);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) a[e] = g[e] = 0u;
+        }
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint4 wv, wk;
+          wv.x = pack_bf16x2(__uint_as_float(a[c8 * 8 + 0]), __uint_as_float(a[c8 * 8 + 1]));
+          wv.y = pack_bf16x2(__uint_as_float(a[c8 * 8 + 2]), __uint_as_float(a[c8 * 8 + 3]));
+          wv.z = pack_bf16x2(__uint_as_float(a[c8 * 8 + 4]), __uint_as_float(a[c8 * 8 + 5]));
+          wv.w = pack_bf16x2(__uint_as_float(a[c8 * 8 + 6]), __uint_as_float(a[c8 * 8 + 7]));
+          wk.x = pack_bf16x2(__uint_as_float(g[c8 * 8 + 0]) * p.scale, __uint_as_float(g[c8 * 8 + 1]) * p.scale);
+          wk.y = pack_bf16x2(__uint_as_float(g[c8 * 8 + 2]) * p.scale, __uint_as_float(g[c8 * 8 + 3]) * p.scale);
+          wk.z = pack_bf16x2(__uint_as_float(g[c8 * 8 + 4]) * p.scale, __uint_as_float(g[c8 * 8 + 5]) * p.scale);
+          wk.w = pack_bf16x2(__uint_as_float(g[c8 * 8 + 6]) * p.scale, __uint_as_float(g[c8 * 8 + 7]) * p.scale);
+          if (j < p.Sk) {
+            *reinterpret_cast<uint4*>(p.dv + row + q * 32 + c8 * 8) = wv;
+            *reinterpret_cast<uint4*>(p.dk + row + q * 32 + c8 * 8) = wk;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------- dQ kernel
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+  using Cfg = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // Q | dO | stage 0: K, V (vector space unused) | stage 1 | barriers
+  const uint32_t sQ = smem_u32(smem);
+  const uint32_t sDO = sQ + Cfg::kTileBytes;
+  auto sK = [&](int st) { return sQ + 2 * Cfg::kTileBytes + st * Cfg::kStageBytes; };
+  auto sV = [&](int st) { return sK(st) + Cfg::kTileBytes; };
+  const uint32_t bar0 = sQ + 2 * Cfg::kTileBytes + kBwdStages * Cfg::kStageBytes;
+  const uint32_t res_full = bar0;
+  auto st_full = [&](int st) { return bar0 + 8u * (1 + st); };
+  auto st_empty = [&](int st) { return bar0 + 8u * (1 + kBwdStages + st); };
+  const uint32_t s_full = bar0 + 8u * (1 + 2 * kBwdStages);
+  const uint32_t p_full = s_full + 8u;
+  const uint32_t done = p_full + 8u;
+  uint8_t* bar_ptr = smem + 2 * Cfg::kTileBytes + kBwdStages * Cfg::kStageBytes;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * Cfg::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int qt = static_cast<int>(blockIdx.x % p.n_qt);
+  const int bh = static_cast<int>(blockIdx.x / p.n_qt);
+  const int b = bh / p.Hq;
+  const int hq = bh - b * p.Hq;
+  const int hkv = hq / p.group;
+  const int i0 = qt * 128;
+  // key tiles this query tile sees: keys j <= last row + coff (causal)
+  int n_it = p.n_kt;
+  if (p.causal) {
+    const int last_key = min(i0 + 127, p.Sq - 1) + p.coff;
+    n_it = last_key < 0 ? 0 : min(p.n_kt, last_key / 128 + 1);
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(res_full, 1);
+    for (int st = 0; st < kBwdStages; ++st) {
+      mbar_init(st_full(st), 1);
+      mbar_init(st_empty(st), 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM columns: S [0,128) | dP [128,256) | dQ [256,256+D)
+  constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
+
+  if (warp == kBwdLoadWarp) {
+    if (lane == 0 && n_it > 0) {
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      mbar_arrive_expect_tx(res_full, 2 * Cfg::kTileBytes);
+      for (int blk = 0; blk < Cfg::kBlocks; ++blk) {
+        tma_load_4d(sQ + blk * Cfg::kBlockBytes, &p.tm_q, blk * 64, i0, hq, b, res_full);
+        tma_load_4d(sDO + blk * Cfg::kBlockBytes, &p.tm_do, blk * 64, i0, hq, b, res_full);
+      }
+      int it = 0;
+      for (; it < n_it; ++it) {
+        const int st = it % kBwdStages;
+        if (!mbar_wait(st_empty(st), ((it / kBwdStages) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(st_full(st), 2 * Cfg::kTileBytes);
+        for (int blk = 0; blk < Cfg::kBlocks; ++blk) {
+          tma_load_4d(sK(st) + blk * Cfg::kBlockBytes, &p.tm_k, blk * 64, it * 128, hkv, b, st_full(st));
+          tma_load_4d(sV(st) + blk * Cfg::kBlockBytes, &p.tm_v, blk * 64, it * 128, hkv, b, st_full(st));
+        }
+      }
+      mbar_wait_drain(res_full, 0);
+      for (int i = max(0, it - kBwdStages); i < it; ++i) mbar_wait_drain(st_full(i % kBwdStages), (i / kBwdStages) & 1);
+    }
+    __syncwarp();
+  } else if (warp == kBwdMmaWarp) {
+    if (lane == 0 && n_it > 0) {
+      const uint64_t hi = static_cast<uint64_t>(sdesc_hi(1024)) << 32;
+      const uint64_t dq_k = hi | sdesc_lo(sQ, 16);
+      const uint64_t ddo_k = hi | sdesc_lo(sDO, 16);
+      bool ok = mbar_wait(res_full, 0, abort_flag);
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int st = it % kBwdStages;
+        if (!mbar_wait(st_full(st), (it / kBwdStages) & 1, abort_flag)) break;
+        tc_fence_after();
+        // S = Q K^T, dP = dO V^T (M = 128 queries, N = 128 keys, K = D)
+        issue_qk<D>(tmem + kColS, dq_k, hi | sdesc_lo(sK(st), 16));
+        issue_qk<D>(tmem + kColDP, ddo_k, hi | sdesc_lo(sV(st), 16));
+        mma_commit(s_full);
+        if (!mbar_wait(p_full, it & 1, abort_flag)) break;
+        tc_fence_after();
+        // dQ += dS K (M = 128 queries, N = D, K = 128 keys; dS from TMEM, K MN-major)
+        const uint64_t dk_mn = hi | sdesc_lo(sK(st), Cfg::kBlockBytes);
+        issue_pv<D, 0>(tmem + kColDQ, tmem + kColS, dk_mn, it > 0);
+        issue_pv<D, 1>(tmem + kColDQ, tmem + kColS, dk_mn, true);
+        mma_commit(st_empty(st));
+      }
+      mma_commit(done);
+      mbar_wait_drain(done, 0);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------ compute: one query row per thread
+    const int r = warp * 32 + lane;
+    const int i = i0 + r;
+    const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+    const float c = p.scale_log2;
+    const int64_t vec = static_cast<int64_t>(bh) * p.Sq_pad + i;
+    const float l2 = __ldg(p.l2 + vec);   // +inf for rows past Sq or that saw no key
+    const float dd = __ldg(p.dvec + vec);
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      // key columns past Sk, or (causal) past row i + coff, are masked
+      const int jlim = min(p.Sk - 1, p.causal ? i + p.coff : INT_MAX) - it * 128;  // last visible column
+      // (warp-uniform: the tcgen05.ld/st below are collective over the warp)
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t sv[32], dp[32];
+        tmem_ld32(tmem + lane_bits + kColS + ch * 32, sv);
+        tmem_ld32(tmem + lane_bits + kColDP + ch * 32, dp);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int col = ch * 32 + e + u;
+            const float pr = (col <= jlim) ? ex2_approx(fmaf(__uint_as_float(sv[e + u]), c, -l2)) : 0.f;
+            ds[u] = pr * (__uint_as_float(dp[e + u]) - dd);
+          }
+          pk[e / 2] = pack_bf16x2(ds[0], ds[1]);
+        }
+        tmem_st16(tmem + lane_bits + kColS + ch * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    // ---- epilogue: dQ = scale * acc -> bf16 row (collective TMEM loads by
+    // the whole warp; only the stores depend on the lane's row)
+    const bool have = __all_sync(0xffffffffu, ok && n_it > 0 && mbar_wait(done, 0, abort_flag));
+    if (have) tc_fence_after();
+    {
+      uint16_t* dst = p.dq + (static_cast<int64_t>(bh) * p.Sq + i) * D;
+#pragma unroll 1
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t a[32];
+        if (have) {
+          tmem_ld32(tmem + lane_bits + kColDQ + q * 32, a);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) a[e] = 0u;
+        }
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(a[c8 * 8 + 0]) * p.scale, __uint_as_float(a[c8 * 8 + 1]) * p.scale);
+          w.y = pack_bf16x2(__uint_as_float(a[c8 * 8 + 2]) * p.scale, __uint_as_float(a[c8 * 8 + 3]) * p.scale);
+          w.z = pack_bf16x2(__uint_as_float(a[c8 * 8 + 4]) * p.scale, __uint_as_float(a[c8 * 8 + 5]) * p.scale);
+          w.w = pack_bf16x2(__uint_as_float(a[c8 * 8 + 6]) * p.scale, __uint_as_float(a[c8 * 8 + 7]) * p.scale);
+          if (i < p.Sq) *reinterpret_cast<uint4*>(dst + q * 32 + c8 * 8) = w;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace sdpa

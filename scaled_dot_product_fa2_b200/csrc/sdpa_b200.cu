@@ -15,6 +15,7 @@
 #include "decode.cuh"
 #include "prefill.cuh"
 #include "rope.cuh"
+#include "backward.cuh"
 
 namespace sdpa {
 constexpr int kMaxDeviceSlots = 64;
@@ -202,6 +203,20 @@ attn_status_t launch_fill_empty(void* o, float* lse, int64_t rows, int d, cudaSt
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Fill a bf16 buffer with zeros (gradients of inputs no row depends on).
+__global__ void fill_zero_kernel(uint16_t* x, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    x[i] = 0;
+}
+
+attn_status_t launch_fill_zero(void* x, int64_t n, cudaStream_t st) {
+  if (n <= 0) return ATTN_OK;
+  const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096));
+  fill_zero_kernel<<<blocks, 256, 0, st>>>(static_cast<uint16_t*>(x), n);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 template <int D, int NS, bool BIAS>
 attn_status_t launch_prefill(const PrefillParams& prm, int grid, int dev, cudaStream_t st) {
   static bool smem_done[kMaxDevices] = {};
@@ -325,6 +340,36 @@ attn_status_t launch_decode(const DecodeParams& prm, int grid, float* part_o, fl
                             prm.nsplit, ol) == cudaSuccess
              ? ATTN_OK
              : ATTN_ERR_CUDA;
+}
+
+// The three backward kernels, in stream order: prep (D, LSE in log2), then
+// dK/dV over key tiles, then dQ over query tiles.
+template <int D>
+attn_status_t launch_bwd(const BwdParams& prm, int dev, cudaStream_t st) {
+  static bool smem_done_kv[kMaxDevices] = {};
+  static bool smem_done_q[kMaxDevices] = {};
+  static std::mutex mu;
+  using Cfg = BwdCfg<D>;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!set_smem(bwd_dkdv_kernel<D>, Cfg::kSmemLaunch, dev, smem_done_kv) ||
+        !set_smem(bwd_dq_kernel<D>, Cfg::kSmemLaunch, dev, smem_done_q))
+      return ATTN_ERR_CUDA;
+  }
+  const int64_t prep_rows = static_cast<int64_t>(prm.B) * prm.Hq * prm.Sq_pad;
+  bwd_prep_kernel<D><<<static_cast<unsigned>((prep_rows + 7) / 8), 256, 0, st>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  const int64_t g_kv = static_cast<int64_t>(prm.B) * prm.Hkv * prm.n_kt;
+  const int64_t g_q = static_cast<int64_t>(prm.B) * prm.Hq * prm.n_qt;
+  if (g_kv > 0) {
+    bwd_dkdv_kernel<D><<<static_cast<unsigned>(g_kv), kBwdThreads, Cfg::kSmemLaunch, st>>>(prm);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  if (g_q > 0) {
+    bwd_dq_kernel<D><<<static_cast<unsigned>(g_q), kBwdThreads, Cfg::kSmemLaunch, st>>>(prm);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
 }
 
 // Blocks for the rotary/append kernel: one per token, at most one resident
@@ -537,6 +582,67 @@ attn_status_t attn_decode_splitkv_ex(const void* q, const void* k_cache, const v
                                      const attn_extras_t* extras, void* stream) {
   return decode_impl(q, k_cache, v_cache, extras, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal, num_splits,
                      workspace, workspace_bytes, stream);
+}
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Sq) {
+  if (B < 0 || Hq <= 0 || Sq < 0 || Sq > kMaxSeq) return 0;
+  const int64_t sq_pad = (static_cast<int64_t>(Sq) + 127) / 128 * 128;
+  return static_cast<size_t>(2 * static_cast<int64_t>(B) * Hq * sq_pad * 4);
+}
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                       float scale, int causal, void* workspace, size_t workspace_bytes, void* stream) {
+  attn_status_t s = check_common(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
+  if (s != ATTN_OK) return s;
+  if (B == 0) return ATTN_OK;
+  const bool have_q = Sq > 0, have_k = Sk > 0;
+  if (have_q && (dq == nullptr || dout == nullptr)) return ATTN_ERR_NULL;
+  if (have_k && (dk == nullptr || dv == nullptr || k == nullptr || v == nullptr)) return ATTN_ERR_NULL;
+  if ((have_q && (!aligned(dq, 16) || !aligned(dout, 16))) || (have_k && (!aligned(dk, 16) || !aligned(dv, 16))))
+    return ATTN_ERR_ALIGN;
+  int dev = 0, sms = 0;
+  if ((s = current_device(&dev, &sms)) != ATTN_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // no query rows: nothing depends on k, v; no keys: o = 0 does not depend on q
+  if (!have_q) return launch_fill_zero(dk, static_cast<int64_t>(B) * Hkv * Sk * d, st) == ATTN_OK
+                          ? launch_fill_zero(dv, static_cast<int64_t>(B) * Hkv * Sk * d, st)
+                          : ATTN_ERR_CUDA;
+  if (!have_k) return launch_fill_zero(dq, static_cast<int64_t>(B) * Hq * Sq * d, st);
+  if (lse == nullptr || o == nullptr) return ATTN_ERR_NULL;
+  const size_t need = attn_bwd_workspace_size(B, Hq, Sq);
+  if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16)) return ATTN_ERR_WORKSPACE;
+
+  BwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  if (!make_map4(&prm.tm_q, q, ATTN_LAYOUT_BHSD, B, Hq, Sq, d, 128) ||
+      !make_map4(&prm.tm_k, k, ATTN_LAYOUT_BHSD, B, Hkv, Sk, d, 128) ||
+      !make_map4(&prm.tm_v, v, ATTN_LAYOUT_BHSD, B, Hkv, Sk, d, 128) ||
+      !make_map4(&prm.tm_do, dout, ATTN_LAYOUT_BHSD, B, Hq, Sq, d, 128))
+    return ATTN_ERR_CUDA;
+  const int sq_pad = (Sq + 127) / 128 * 128;
+  prm.o = static_cast<const uint16_t*>(o);
+  prm.dout = static_cast<const uint16_t*>(dout);
+  prm.lse = lse;
+  prm.l2 = static_cast<float*>(workspace);
+  prm.dvec = prm.l2 + static_cast<int64_t>(B) * Hq * sq_pad;
+  prm.dq = static_cast<uint16_t*>(dq);
+  prm.dk = static_cast<uint16_t*>(dk);
+  prm.dv = static_cast<uint16_t*>(dv);
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.Sq = Sq;
+  prm.Sk = Sk;
+  prm.Sq_pad = sq_pad;
+  prm.group = Hq / Hkv;
+  prm.causal = causal;
+  prm.coff = causal_offset(causal, Sq, Sk);
+  prm.n_qt = sq_pad / 128;
+  prm.n_kt = (Sk + 127) / 128;
+  prm.scale = effective_scale(scale, d);
+  prm.scale_log2 = prm.scale * 1.4426950408889634f;
+  return d == 128 ? launch_bwd<128>(prm, dev, st) : launch_bwd<64>(prm, dev, st);
 }
 
 attn_status_t attn_rope_append(const void* packed_qkv, const float* cos_table, const float* sin_table, int max_pos,

@@ -264,6 +264,42 @@ def attn_decode_splitkv_static(q, k_cache, v_cache, causal: int = CAUSAL_BOTTOM_
     return out, lse
 
 
+def attn_bwd(q, k, v, o, lse, dout, causal: int = CAUSAL_NONE, scale: float = 0.0, dq=None, dk=None, dv=None,
+             workspace=None):
+    """Gradients (dq, dk, dv) of the forward ``o, lse = attn_fwd(q, k, v, causal, scale)``
+    for ``dout`` = dL/do (``attn_bwd``).  BHSD tensors, bf16; lse fp32 from the forward.
+
+    P is recomputed from ``lse``; nothing of size Sq x Sk is stored.  dk and dv
+    of a KV head sum over the query heads that share it.
+    """
+    B, Hq, Hkv, Sq, Sk, d = _shapes(q, k, v)
+    _check_tensor("o", o, torch.bfloat16, 4)
+    _check_tensor("dout", dout, torch.bfloat16, 4)
+    _check_tensor("lse", lse, torch.float32, 3)
+    if tuple(o.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("o and dout must have q's shape")
+    if tuple(lse.shape) != (B, Hq, Sq):
+        raise ValueError("lse must be [B, Hq, Sq]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t, ref in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        _check_tensor(name, t, torch.bfloat16, 4)
+        if tuple(t.shape) != tuple(ref.shape) or t.device != q.device:
+            raise ValueError(f"{name} must match {tuple(ref.shape)} on q's device")
+    lib = _lib.get()
+    need = int(lib.attn_bwd_workspace_size(B, Hq, Sq))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Sq, Sk, d, float(scale),
+                          int(causal), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                          _stream_handle(q.device))
+    _lib.check(st, "attn_bwd")
+    return dq, dk, dv
+
+
 def attn_rope_append(packed_qkv, cos, sin, past_lens, k_cache, v_cache, Hq: int, Hkv: int,
                      layout: int = LAYOUT_BHSD, q_out=None, total_lens=None):
     """Split a packed QKV projection, rotate q and k, append k and v to the cache

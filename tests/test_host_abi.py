@@ -207,3 +207,22 @@ def test_rope_append_rejects_bad_arguments_on_host(lib):
     # nothing to do: no batch, or no new token and no total lengths wanted
     assert call(B=0, packed=None, cos=None, sin=None, past=None, q=None, kc=None, vc=None, tot=None) == 0
     assert call(S_new=0, packed=None, cos=None, sin=None, q=None, kc=None, vc=None, tot=None) == 0
+
+
+def test_bwd_rejects_bad_arguments_on_host(lib):
+    need = lib.attn_bwd_workspace_size(2, 4, 100)
+    assert need == 2 * 2 * 4 * 128 * 4  # rows padded to whole 128-row tiles, two fp32 vectors
+    assert lib.attn_bwd_workspace_size(-1, 4, 100) == 0
+
+    def call(q=P, k=P, v=P, o=P, lse=P, do=P, dq=P, dk=P, dv=P, B=2, Hq=4, Hkv=2, Sq=100, Sk=90, d=128,
+             scale=0.0, causal=0, ws=P, wsb=None):
+        return lib.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d, scale, causal, ws,
+                            need if wsb is None else wsb, None)
+    for kw, status in [
+        (dict(q=None), 1), (dict(o=None), 1), (dict(dq=None), 1), (dict(do=None), 1), (dict(dk=None), 1),
+        (dict(dv=None), 1), (dict(B=-1), 2), (dict(Hq=6, Hkv=4), 3), (dict(d=96), 4),
+        (dict(dq=P + 8), 5), (dict(dk=P + 2), 5), (dict(do=P + 4), 5), (dict(causal=3), 6),
+        (dict(scale=-1.0), 11),
+    ]:
+        assert call(**kw) == status, kw
+    assert call(B=0, q=None, k=None, v=None, o=None, lse=None, do=None, dq=None, dk=None, dv=None, ws=None) == 0
