@@ -640,6 +640,10 @@ def run_profile_case(args):
     if args.profile in rope:
         w = rope[args.profile]
         runner = GpuRopeAppend(w, 0)
+    elif args.profile.startswith("bwd_"):
+        # the backward pass of a prefill workload, e.g. bwd_prefill_noncausal_s4096
+        w = inputs.BY_NAME[args.profile[len("bwd_"):]]
+        runner = GpuBackward(w, 0)
     else:
         w = inputs.BY_NAME[args.profile]
         runner = GpuDecode(w, 0) if w.decode else GpuPrefill(w, 0)
