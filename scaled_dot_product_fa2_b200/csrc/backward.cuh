@@ -18,13 +18,17 @@
 //                     stay in shared memory while the query tiles of every
 //                     query head of the group stream through a 2-stage ring.
 //                     Per query tile: S^T = K Q^T and dP^T = V dO^T (tcgen05,
-//                     into TMEM), P^T and dS^T by the four compute warps (one
-//                     thread per key row, written back to TMEM as bf16 over
-//                     the first half of S^T and dP^T), then dV += P^T dO and
+//                     into TMEM), P^T and dS^T by eight compute warps (two per
+//                     key row, one for each half of the 128 query columns;
+//                     each half's bf16 results overwrite that half's first
+//                     32 columns of S^T and dP^T), then dV += P^T dO and
 //                     dK += dS^T Q with P^T, dS^T read from TMEM.
 //   bwd_dq_kernel     one CTA per 128-row query tile: Q and dO stay in shared
 //                     memory while the key tiles stream; S = Q K^T and
-//                     dP = dO V^T, dS by the compute warps, dQ += dS K.
+//                     dP = dO V^T, dS by the compute warps into TMEM columns
+//                     of its own, dQ += dS K.  With dS apart from S, the next
+//                     tile's S and dP are issued before this tile's dS K, so
+//                     the compute warps wait for two matmuls a tile, not three.
 // Fully masked key tiles are skipped (causal).  TMEM holds every accumulator
 // (dK and dV for the whole query loop, dQ for the whole key loop).  Every
 // wait is bounded; a timeout sets the device error word and the kernel exits.
@@ -55,9 +59,10 @@ struct BwdParams {
   float scale_log2;  // scale * log2(e)
 };
 
-constexpr int kBwdThreads = 192;  // warps 0-3 compute, 4 MMA issuer (+ TMEM owner), 5 TMA producer
-constexpr int kBwdMmaWarp = 4;
-constexpr int kBwdLoadWarp = 5;
+constexpr int kBwdThreads = 320;  // warps 0-7 compute, 8 MMA issuer (+ TMEM owner), 9 TMA producer
+constexpr int kBwdComputeWarps = 8;
+constexpr int kBwdMmaWarp = 8;
+constexpr int kBwdLoadWarp = 9;
 constexpr int kBwdStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -88,8 +93,9 @@ struct BwdCfg {
   static constexpr int kVecBytes = 128 * 4;         // 128 fp32 (L2 or D of one query tile)
   // smem: two resident tiles, then per stage two streamed tiles and two vectors
   static constexpr int kStageBytes = 2 * kTileBytes + 2 * kVecBytes;
-  // res_full, st_full[2], st_empty[2], s_full, p_full, done
-  static constexpr int kNumBars = 1 + 2 * kBwdStages + 3;
+  // res_full, st_full[2], st_empty[2], s_full, p_full, done, ds_free (dQ only: the
+  // previous dS has been read)
+  static constexpr int kNumBars = 1 + 2 * kBwdStages + 4;
   static constexpr int kSmemBytes = 2 * kTileBytes + kBwdStages * kStageBytes + kNumBars * 8 + 16 + 1024;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
   static constexpr uint32_t kTmemCols = 512;
@@ -126,6 +132,32 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __grid_constant__ B
   if (lane == 0) {
     p.dvec[w] = dsum;
     p.l2[w] = l2;
+  }
+}
+
+// P^T and dS^T for 32 query columns col0 .. col0+31 of one key row: sv, dp
+// hold S^T and dP^T, l2v / ddv the query tile's LSE*log2(e) and D; columns
+// before cmin do not see the key.  Results as bf16 pairs.
+__device__ __forceinline__ void dkdv_chunk(const uint32_t (&sv)[32], const uint32_t (&dp)[32], const float* l2v,
+                                           const float* ddv, int col0, int cmin, float c, uint32_t (&pk)[16],
+                                           uint32_t (&dk16)[16]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) {
+    const float4 lv = *reinterpret_cast<const float4*>(l2v + col0 + e);
+    const float4 dv4 = *reinterpret_cast<const float4*>(ddv + col0 + e);
+    const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
+    const float dq4[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+    float pr[4], ds[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float x = fmaf(__uint_as_float(sv[e + u]), c, -lq[u]);
+      pr[u] = (col0 + e + u >= cmin) ? ex2_approx(x) : 0.f;
+      ds[u] = pr[u] * (__uint_as_float(dp[e + u]) - dq4[u]);
+    }
+    pk[e / 2] = pack_bf16x2(pr[0], pr[1]);
+    pk[e / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
+    dk16[e / 2] = pack_bf16x2(ds[0], ds[1]);
+    dk16[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
   }
 }
 
@@ -173,7 +205,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       mbar_init(st_empty(st), 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);  // one arrive per compute warp
+    mbar_init(p_full, kBwdComputeWarps);  // one arrive per compute warp
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -240,21 +272,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         // A from TMEM, B = the query-side tile, MN-major).
         const uint64_t ddo_mn = hi | sdesc_lo(sDO(st), Cfg::kBlockBytes);
         const uint64_t dq_mn = hi | sdesc_lo(sQ(st), Cfg::kBlockBytes);
+        // P^T, dS^T of queries 0..63 are at columns 0..31 of S^T / dP^T and of
+        // queries 64..127 at 64..95: issue_pv reads keys 16 kk.. at column 8 kk
+        // of its base, so the second half's base is 32 columns further.
         issue_pv<D, 0>(tmem + kColDV, tmem + kColS, ddo_mn, it > 0);
-        issue_pv<D, 1>(tmem + kColDV, tmem + kColS, ddo_mn, true);
+        issue_pv<D, 1>(tmem + kColDV, tmem + kColS + 32, ddo_mn, true);
         issue_pv<D, 0>(tmem + kColDK, tmem + kColDP, dq_mn, it > 0);
-        issue_pv<D, 1>(tmem + kColDK, tmem + kColDP, dq_mn, true);
+        issue_pv<D, 1>(tmem + kColDK, tmem + kColDP + 32, dq_mn, true);
         mma_commit(st_empty(st));
       }
       mma_commit(done);
       mbar_wait_drain(done, 0);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ------------------------------------------------ compute: one key row per thread
-    const int r = warp * 32 + lane;
+  } else if (warp < kBwdComputeWarps) {
+    // ------------------------------------ compute: two warps per key row (column halves)
+    // Warpgroup wg takes query columns 64 wg .. 64 wg + 63 (chunks 2 wg, 2 wg + 1)
+    // of TMEM lane quarter `quarter` and writes their bf16 results over its
+    // own first 32 columns (64 wg .. 64 wg + 31 of S^T and of dP^T), which it
+    // has already read: the two warpgroups never touch each other's columns.
+    // The dV/dK MMAs read queries 0..63 at column 0 and 64..127 at column 64.
+    const int wg = warp >> 2;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
     const int j = k0 + r;
-    const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_bits + kColS + 64 * wg;
+    const uint32_t tDP = tmem + lane_bits + kColDP + 64 * wg;
     const float c = p.scale_log2;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
@@ -263,8 +307,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       // query columns c < cmin do not see key j (causal); keys past Sk see nothing
       const int cmin = (j >= p.Sk) ? INT_MAX : (p.causal ? j - p.coff - qt * 128 : INT_MIN);
       // S^T/dP^T ready; the stage's L2/D vectors landed (the wait on the
-      // stage's own barrier makes the bulk copy's writes visible here)
-      // (warp-uniform: the tcgen05.ld/st below are collective over the warp)
+      // stage's own barrier makes the bulk copy's writes visible here).
+      // Warp-uniform: the tcgen05.ld/st below are collective over the warp.
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag) &&
                                        mbar_wait(st_full(st), (it / kBwdStages) & 1, abort_flag));
       if (!ok) break;
@@ -272,35 +316,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       const float* l2v = l2_at(st);
       const float* ddv = dd_at(st);
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t sv[32], dp[32];
-        tmem_ld32(tmem + lane_bits + kColS + ch * 32, sv);
-        tmem_ld32(tmem + lane_bits + kColDP + ch * 32, dp);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t sv[32], dp[32], pk[16], dk16[16];
+        tmem_ld32(tS + 32 * h, sv);
+        tmem_ld32(tDP + 32 * h, dp);
         tmem_wait_ld();
-        uint32_t pk[16], dk16[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 lv = *reinterpret_cast<const float4*>(l2v + ch * 32 + e);
-          const float4 dv4 = *reinterpret_cast<const float4*>(ddv + ch * 32 + e);
-          const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
-          const float dq4[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
-          float pr[4], ds[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int col = ch * 32 + e + u;
-            const float x = fmaf(__uint_as_float(sv[e + u]), c, -lq[u]);
-            pr[u] = (col >= cmin) ? ex2_approx(x) : 0.f;
-            ds[u] = pr[u] * (__uint_as_float(dp[e + u]) - dq4[u]);
-          }
-          pk[e / 2] = pack_bf16x2(pr[0], pr[1]);
-          pk[e / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
-          dk16[e / 2] = pack_bf16x2(ds[0], ds[1]);
-          dk16[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
-        }
-        // chunk ch of S^T / dP^T is in registers; its bf16 result goes to
-        // columns already read (16 ch .. 16 ch + 15)
-        tmem_st16(tmem + lane_bits + kColS + ch * 16, pk);
-        tmem_st16(tmem + lane_bits + kColDP + ch * 16, dk16);
+        dkdv_chunk(sv, dp, l2v, ddv, 64 * wg + 32 * h, cmin, c, pk, dk16);
+        // columns 16 h .. 16 h + 15 of this half: read in step 0 already
+        tmem_st16(tS + 16 * h, pk);
+        tmem_st16(tDP + 16 * h, dk16);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -315,7 +339,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     {
       const int64_t row = ((static_cast<int64_t>(b) * p.Hkv + hkv) * p.Sk + j) * D;
 #pragma unroll 1
-      for (int q = 0; q < D / 32; ++q) {
+      for (int q = wg * (D / 64); q < (wg + 1) * (D / 64); ++q) {  // this warpgroup's half of the columns
         uint32_t a[32], g[32];
         if (have) {
           tmem_ld32(tmem + lane_bits + kColDV + q * 32, a);
@@ -371,6 +395,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
   const uint32_t s_full = bar0 + 8u * (1 + 2 * kBwdStages);
   const uint32_t p_full = s_full + 8u;
   const uint32_t done = p_full + 8u;
+  const uint32_t ds_free = done + 8u;  // dQ += dS K of the previous key tile is done
   uint8_t* bar_ptr = smem + 2 * Cfg::kTileBytes + kBwdStages * Cfg::kStageBytes;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * Cfg::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -397,8 +422,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       mbar_init(st_empty(st), 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, kBwdComputeWarps);
     mbar_init(done, 1);
+    mbar_init(ds_free, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -410,8 +436,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM columns: S [0,128) | dP [128,256) | dQ [256,256+D)
-  constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
+  // TMEM columns: S [0,128) | dP [128,256) | dQ [256,256+D) | dS [384,448) (bf16 pairs)
+  constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColDS = 384;
 
   if (warp == kBwdLoadWarp) {
     if (lane == 0 && n_it > 0) {
@@ -441,32 +467,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       const uint64_t hi = static_cast<uint64_t>(sdesc_hi(1024)) << 32;
       const uint64_t dq_k = hi | sdesc_lo(sQ, 16);
       const uint64_t ddo_k = hi | sdesc_lo(sDO, 16);
-      bool ok = mbar_wait(res_full, 0, abort_flag);
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int st = it % kBwdStages;
-        if (!mbar_wait(st_full(st), (it / kBwdStages) & 1, abort_flag)) break;
-        tc_fence_after();
-        // S = Q K^T, dP = dO V^T (M = 128 queries, N = 128 keys, K = D)
+      auto issue_s_dp = [&](int st) {  // S = Q K^T, dP = dO V^T (M = 128 queries, N = 128 keys, K = D)
         issue_qk<D>(tmem + kColS, dq_k, hi | sdesc_lo(sK(st), 16));
         issue_qk<D>(tmem + kColDP, ddo_k, hi | sdesc_lo(sV(st), 16));
         mma_commit(s_full);
-        if (!mbar_wait(p_full, it & 1, abort_flag)) break;
+      };
+      bool ok = mbar_wait(res_full, 0, abort_flag) && mbar_wait(st_full(0), 0, abort_flag);
+      if (ok) {
         tc_fence_after();
+        issue_s_dp(0);
+      }
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int st = it % kBwdStages;
+        // dS(it) written (S, dP of tile it no longer needed), next tile landed
+        if (!mbar_wait(p_full, it & 1, abort_flag)) break;
+        const bool next = it + 1 < n_it;
+        if (next && !mbar_wait(st_full((it + 1) % kBwdStages), ((it + 1) / kBwdStages) & 1, abort_flag)) break;
+        tc_fence_after();
+        if (next) issue_s_dp((it + 1) % kBwdStages);
         // dQ += dS K (M = 128 queries, N = D, K = 128 keys; dS from TMEM, K MN-major)
         const uint64_t dk_mn = hi | sdesc_lo(sK(st), Cfg::kBlockBytes);
-        issue_pv<D, 0>(tmem + kColDQ, tmem + kColS, dk_mn, it > 0);
-        issue_pv<D, 1>(tmem + kColDQ, tmem + kColS, dk_mn, true);
+        issue_pv<D, 0>(tmem + kColDQ, tmem + kColDS, dk_mn, it > 0);
+        issue_pv<D, 1>(tmem + kColDQ, tmem + kColDS, dk_mn, true);
+        mma_commit(ds_free);
         mma_commit(st_empty(st));
       }
       mma_commit(done);
       mbar_wait_drain(done, 0);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ------------------------------------------------ compute: one query row per thread
-    const int r = warp * 32 + lane;
+  } else if (warp < kBwdComputeWarps) {
+    // ------------------------------------ compute: two warps per query row (column halves)
+    const int wg = warp >> 2;  // key columns 64 wg .. 64 wg + 63
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
     const int i = i0 + r;
-    const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
     const float c = p.scale_log2;
     const int64_t vec = static_cast<int64_t>(bh) * p.Sq_pad + i;
     const float l2 = __ldg(p.l2 + vec);   // +inf for rows past Sq or that saw no key
@@ -479,13 +515,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
+      uint32_t pk[2][16];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int ch = 2 * wg + h;
         uint32_t sv[32], dp[32];
         tmem_ld32(tmem + lane_bits + kColS + ch * 32, sv);
         tmem_ld32(tmem + lane_bits + kColDP + ch * 32, dp);
         tmem_wait_ld();
-        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           float ds[2];
@@ -495,10 +532,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             const float pr = (col <= jlim) ? ex2_approx(fmaf(__uint_as_float(sv[e + u]), c, -l2)) : 0.f;
             ds[u] = pr * (__uint_as_float(dp[e + u]) - dd);
           }
-          pk[e / 2] = pack_bf16x2(ds[0], ds[1]);
+          pk[h][e / 2] = pack_bf16x2(ds[0], ds[1]);
         }
-        tmem_st16(tmem + lane_bits + kColS + ch * 16, pk);
       }
+      // the dS columns are free once dQ += dS K of the previous key tile is done
+      if (it > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(ds_free, (it - 1) & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      tmem_st16(tmem + lane_bits + kColDS + (2 * wg) * 16, pk[0]);
+      tmem_st16(tmem + lane_bits + kColDS + (2 * wg + 1) * 16, pk[1]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -511,7 +555,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
     {
       uint16_t* dst = p.dq + (static_cast<int64_t>(bh) * p.Sq + i) * D;
 #pragma unroll 1
-      for (int q = 0; q < D / 32; ++q) {
+      for (int q = wg * (D / 64); q < (wg + 1) * (D / 64); ++q) {  // this warpgroup's half of the columns
         uint32_t a[32];
         if (have) {
           tmem_ld32(tmem + lane_bits + kColDQ + q * 32, a);
