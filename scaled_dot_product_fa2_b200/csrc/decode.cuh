@@ -219,7 +219,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
 
   for (int it = 0; it < ntiles; ++it) {
     const int st = it % NSTAGE;
-    if (!mbar_wait(full(st), (it / NSTAGE) & 1, abort_flag)) {
+    // warp-uniform: a lane that gave up must not leave its warp's mma.sync
+    if (!__all_sync(0xffffffffu, mbar_wait(full(st), (it / NSTAGE) & 1, abort_flag))) {
       ok = false;
       break;
     }
