@@ -348,8 +348,7 @@ class GpuBackward(GpuPrefill):
         self.dq = torch.empty_like(self.q)
         self.dk = torch.empty_like(self.k)
         self.dv = torch.empty_like(self.v)
-        self.ws = torch.empty(max(16, sdpa.ops._lib.get().attn_bwd_workspace_size(w.B, w.Hq, w.Sq)),
-                              dtype=torch.uint8, device="cuda")
+        self.ws = torch.empty(max(16, sdpa.bwd_workspace_size(w.B, w.Hq, w.Sq)), dtype=torch.uint8, device="cuda")
 
     def run(self):
         import scaled_dot_product_fa2_b200 as sdpa

@@ -153,6 +153,11 @@ def decode_workspace_size(B, Hq, Hkv, Sq, Sk, d, num_splits: int = 0) -> int:
     return int(_lib.get().attn_decode_workspace_size(B, Hq, Hkv, Sq, Sk, d, num_splits))
 
 
+def bwd_workspace_size(B, Hq, Sq) -> int:
+    """Bytes of workspace ``attn_bwd`` needs (``attn_bwd_workspace_size``)."""
+    return int(_lib.get().attn_bwd_workspace_size(B, Hq, Sq))
+
+
 def decode_workspace(q, k_cache, num_splits: int = 0) -> torch.Tensor:
     """A caller-owned workspace buffer sized for ``attn_decode_splitkv``."""
     B, Hq, Sq, d = q.shape
@@ -288,9 +293,8 @@ def attn_bwd(q, k, v, o, lse, dout, causal: int = CAUSAL_NONE, scale: float = 0.
         if tuple(t.shape) != tuple(ref.shape) or t.device != q.device:
             raise ValueError(f"{name} must match {tuple(ref.shape)} on q's device")
     lib = _lib.get()
-    need = int(lib.attn_bwd_workspace_size(B, Hq, Sq))
     if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(max(bwd_workspace_size(B, Hq, Sq), 16), dtype=torch.uint8, device=q.device)
     with torch.cuda.device(q.device):
         st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Sq, Sk, d, float(scale),

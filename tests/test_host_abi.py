@@ -226,3 +226,20 @@ def test_bwd_rejects_bad_arguments_on_host(lib):
     ]:
         assert call(**kw) == status, kw
     assert call(B=0, q=None, k=None, v=None, o=None, lse=None, do=None, dq=None, dk=None, dv=None, ws=None) == 0
+
+
+def test_python_entry_points_refuse_host_tensors(lib):
+    """The binding has no CPU path: host tensors are rejected before any call."""
+    import torch
+    import scaled_dot_product_fa2_b200 as sdpa
+    assert sdpa.bwd_workspace_size(2, 4, 100) == lib.attn_bwd_workspace_size(2, 4, 100)
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 2, 8)
+    with pytest.raises(ValueError, match="CUDA"):
+        sdpa.attn_fwd(q, q, q)
+    with pytest.raises(ValueError, match="CUDA"):
+        sdpa.attn_bwd(q, q, q, q, lse, q)
+    packed = torch.zeros(1, 1, 4 * 64, dtype=torch.bfloat16)
+    cos = torch.zeros(8, 32)
+    with pytest.raises(ValueError, match="CUDA"):
+        sdpa.attn_rope_append(packed, cos, cos, torch.zeros(1, dtype=torch.int32), q[:, :1], q[:, :1], 2, 1)
