@@ -243,3 +243,20 @@ def test_python_entry_points_refuse_host_tensors(lib):
     cos = torch.zeros(8, 32)
     with pytest.raises(ValueError, match="CUDA"):
         sdpa.attn_rope_append(packed, cos, cos, torch.zeros(1, dtype=torch.int32), q[:, :1], q[:, :1], 2, 1)
+
+
+@pytest.mark.parametrize("compiler,flags", [("gcc", ["-x", "c", "-std=c99"]), ("g++", ["-x", "c++", "-std=c++17"])])
+def test_header_compiles_as_c_and_cpp(tmp_path, compiler, flags):
+    """The boundary is a C ABI: the header must stand alone in a plain C99
+    translation unit (no CUDA or torch headers needed) and in C++."""
+    import shutil
+    import subprocess
+    if shutil.which(compiler) is None:
+        pytest.skip(f"{compiler} not found")
+    src = tmp_path / "use_header.src"
+    src.write_text('#include "sdpa_b200.h"\n'
+                   'int main(void) { return sizeof(attn_extras_t) > 0 && attn_version() > 0 && '
+                   'attn_status_string(ATTN_OK) != 0 ? 0 : 1; }\n')
+    r = subprocess.run([compiler, *flags, "-Wall", "-Wextra", "-Werror", "-fsyntax-only",
+                        "-I", os.path.dirname(HEADER), str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
