@@ -63,14 +63,14 @@ def _outputs(q, out, lse, want_lse, layout=LAYOUT_BHSD):
         out = torch.empty_like(q)
     else:
         _check_tensor("out", out, torch.bfloat16, 4)
-        if tuple(out.shape) != tuple(q.shape):
-            raise ValueError("out must have the shape of q")
+        if tuple(out.shape) != tuple(q.shape) or out.device != q.device:
+            raise ValueError("out must have the shape of q, on q's device")
     if lse is None and want_lse:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
     elif lse is not None:
         _check_tensor("lse", lse, torch.float32, 3)
-        if tuple(lse.shape) != (B, Hq, Sq):
-            raise ValueError("lse must be [B, Hq, Sq]")
+        if tuple(lse.shape) != (B, Hq, Sq) or lse.device != q.device:
+            raise ValueError("lse must be [B, Hq, Sq] on q's device")
     return out, lse
 
 
@@ -285,6 +285,8 @@ def attn_bwd(q, k, v, o, lse, dout, causal: int = CAUSAL_NONE, scale: float = 0.
         raise ValueError("o and dout must have q's shape")
     if tuple(lse.shape) != (B, Hq, Sq):
         raise ValueError("lse must be [B, Hq, Sq]")
+    if not (o.device == dout.device == lse.device == q.device):
+        raise ValueError("o, lse and dout must be on q's device")
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
