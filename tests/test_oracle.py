@@ -568,3 +568,19 @@ def test_bwd_masked_rows_and_unseen_keys_get_no_gradient(oracle_mod):
     q, k, v, g = _bwd_inputs(1, 1, 1, 3, 6, 4, 141)
     dq, dk, dv = oracle_mod.attn_bwd(q, k, v, g, 0.5, 1)
     assert np.array_equal(dk[0, 0, 3:], np.zeros((3, 4))) and np.array_equal(dv[0, 0, 3:], np.zeros((3, 4)))
+
+
+def test_bwd_two_key_closed_form(oracle_mod):
+    """One query, two keys, d = 1, derived by hand: with x_j = s q k_j,
+    P = softmax(x), o = P1 v1 + P2 v2 and dout = g,
+      dv_j = P_j g,  dx_1 = -dx_2 = P1 P2 g (v1 - v2),
+      dq = s dx_1 (k1 - k2),  dk_1 = -dk_2 = s dx_1 q."""
+    q, k1, k2, v1, v2, g, s = 0.7, -1.3, 0.4, 2.0, -0.5, 1.7, 0.9
+    e1, e2 = np.exp(s * q * k1), np.exp(s * q * k2)
+    P1, P2 = e1 / (e1 + e2), e2 / (e1 + e2)
+    dx1 = P1 * P2 * g * (v1 - v2)
+    dq, dk, dv = oracle_mod.attn_bwd(np.array([[[[q]]]]), np.array([[[[k1], [k2]]]]), np.array([[[[v1], [v2]]]]),
+                                     np.array([[[[g]]]]), s, 0)
+    assert abs(dq[0, 0, 0, 0] - s * dx1 * (k1 - k2)) < 1e-14
+    assert abs(dk[0, 0, 0, 0] - s * dx1 * q) < 1e-14 and abs(dk[0, 0, 1, 0] + s * dx1 * q) < 1e-14
+    assert abs(dv[0, 0, 0, 0] - P1 * g) < 1e-14 and abs(dv[0, 0, 1, 0] - P2 * g) < 1e-14

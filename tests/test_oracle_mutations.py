@@ -62,6 +62,7 @@ def _pin_suite(mod):
     pins.test_bias_of_log_weights_with_zero_query_is_weighted_mean(mod)
     pins.test_bwd_matches_finite_differences(mod, 2, 2, 1, 4, 3, 2, 2)
     pins.test_bwd_single_key_closed_form(mod)
+    pins.test_bwd_two_key_closed_form(mod)
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
