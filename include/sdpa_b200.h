@@ -253,7 +253,10 @@ attn_status_t attn_decode_splitkv_ex(const void* q, const void* k_cache, const v
  *
  * The first call on each device looks up the scratch array's device address
  * (once per device, with that device current); make that first call before
- * any stream capture.  The scratch is shared by every call on a device and
+ * any stream capture.  The address is kept for the life of the process, so a
+ * caller that resets a device (cudaDeviceReset) must not use this entry point
+ * on it afterwards.  On a device that is not a B200 the call returns
+ * ATTN_ERR_ARCH before it looks anything up.  The scratch is shared by every call on a device and
  * keeps the last call's contents; nothing in it needs to start at zero (each
  * call writes every partial it later reads).  Calls that may overlap on the
  * GPU (different streams without ordering between them) race on the scratch:
@@ -314,7 +317,11 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
  *               updated in place: rows past_lens[b] .. past_lens[b] + S_new - 1
  *               receive the rotated k and the unchanged v; no other row is touched.
  *   total_lens  [B] int32, device, or NULL: receives past_lens[b] + S_new, the
- *               key lengths for attn_decode_splitkv_varlen over the updated cache.
+ *               key lengths for attn_decode_splitkv_varlen over the updated cache
+ *               (saturated at INT_MAX).  It may be past_lens itself (lengths
+ *               advanced in place): every token's position is then taken from
+ *               the old lengths, and the new ones are written by a second
+ *               kernel ordered after the append on `stream`.
  *   layout      ATTN_LAYOUT_BHSD or ATTN_LAYOUT_BSHD, for q_out and both caches.
  *
  * All buffers are the caller's; the library allocates nothing.  Pointers must
@@ -329,6 +336,21 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
 attn_status_t attn_rope_append(const void* packed_qkv, const float* cos_table, const float* sin_table, int max_pos,
                                const int* past_lens, void* q_out, void* k_cache, void* v_cache, int* total_lens,
                                int B, int S_new, int Hq, int Hkv, int cap, int d, int layout, void* stream);
+
+/*
+ * Self-test of the bounded-wait contract above (not a computation): runs the
+ * split-KV decode of attn_decode_splitkv (bottom-right mask, default scale,
+ * automatic split count) with its K/V copies withheld, so every consumer
+ * wait in the split kernel gives up after its 1 s limit and the kernel exits
+ * through its timeout path -- no trap, no copy in flight, no tensor memory
+ * held.  The next attn_check_device_error(stream) must then return
+ * ATTN_ERR_DEVICE_TIMEOUT, and the context stays usable.  o and lse receive
+ * meaningless values.  Arguments as for attn_decode_splitkv (B, Sq and Sk
+ * must be > 0); takes about one second of GPU time.
+ */
+attn_status_t attn_selftest_decode_wait_timeout(const void* q, const void* k_cache, const void* v_cache, void* o,
+                                                float* lse, int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                                                void* workspace, size_t workspace_bytes, void* stream);
 
 /* A static, human-readable name for a status code. */
 const char* attn_status_string(attn_status_t status);

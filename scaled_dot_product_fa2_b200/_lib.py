@@ -21,7 +21,7 @@ STATUS_NAMES = {
 STATIC_SCRATCH_BYTES = 16 << 20
 EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_fwd_varlen", "attn_decode_num_splits", "attn_decode_workspace_size", "attn_decode_splitkv",
            "attn_decode_splitkv_varlen", "attn_decode_splitkv_ex", "attn_decode_splitkv_static", "attn_rope_append", "attn_bwd", "attn_bwd_workspace_size",
-           "attn_status_string",
+           "attn_selftest_decode_wait_timeout", "attn_status_string",
            "attn_check_device_error", "attn_version")
 
 class Extras(ctypes.Structure):
@@ -72,6 +72,8 @@ def _declare(lib):
     lib.attn_bwd.restype = I
     lib.attn_bwd_workspace_size.argtypes = [I, I, I]
     lib.attn_bwd_workspace_size.restype = SZ
+    lib.attn_selftest_decode_wait_timeout.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, SZ, P]
+    lib.attn_selftest_decode_wait_timeout.restype = I
     lib.attn_status_string.argtypes = [I]
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_check_device_error.argtypes = [P]

@@ -44,6 +44,8 @@ struct DecodeParams {
   int tiles_per_split;    // 64-key tiles per split
   int row_groups;         // ceil(group*Sq / 16)
   float scale, scale_log2;
+  int withhold_loads;     // self-test only: the producer issues no copy, so every consumer
+                          // wait runs out and the kernel exits through its timeout path
 };
 
 constexpr int kDecKeys = 64;          // keys per tile
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
   __syncthreads();
 
   if (warp == kDecProducerWarp) {
-    if (lane == 0 && ntiles > 0) {
+    if (lane == 0 && ntiles > 0 && !p.withhold_loads) {
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
       int issued = 0;

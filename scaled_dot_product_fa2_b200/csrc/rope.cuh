@@ -20,6 +20,8 @@
 // partner half of each rotated pair sits d/16 lanes away and comes over by
 // shuffle.
 #pragma once
+#include <climits>
+
 #include "ptx.cuh"
 
 namespace sdpa {
@@ -32,7 +34,8 @@ struct RopeParams {
   uint16_t* q_out;         // q rows, element (b, h, t, :) at b*q_sb + h*q_sh + t*q_sr
   uint16_t* k_cache;       // cache rows, element (b, h, pos, :) at b*c_sb + h*c_sh + pos*c_sr
   uint16_t* v_cache;
-  int* total_lens;         // [B] past + S_new, or nullptr
+  int* total_lens;         // [B] past + S_new written by this kernel, or nullptr (none, or
+                           // written by rope_lengths_kernel afterwards when it aliases past_lens)
   int64_t q_sb, q_sh, q_sr;
   int64_t c_sb, c_sh, c_sr;
   int tokens;              // B * S_new (< 2^31, checked on the host)
@@ -42,6 +45,23 @@ struct RopeParams {
 constexpr int kRopeWarps = 8;        // warps per block (256 threads)
 constexpr int kRopeUnroll = 3;       // block passes over a token's head rows with loads in flight together
 constexpr int kRopeBlocksPerSm = 4;  // resident blocks per SM
+
+// past + S_new, saturated to the int range instead of wrapping (a corrupt
+// past near INT_MAX gives INT_MAX, which a later decode clamps and reports).
+__device__ __forceinline__ int rope_total_length(int past, int s_new) {
+  const long long t = static_cast<long long>(past) + s_new;
+  return t > INT_MAX ? INT_MAX : static_cast<int>(t);
+}
+
+// total_lens[b] = past_lens[b] + S_new as a second, stream-ordered step: used
+// when the two arrays overlap (lengths updated in place), so that no block of
+// the append kernel can read a past length another block has already advanced.
+__global__ void rope_lengths_kernel(const int* past_lens, int* total_lens, int B, int s_new) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < B; i += gridDim.x * blockDim.x) {
+    const int past = past_lens[i];  // plain load: the array may be the one written
+    total_lens[i] = rope_total_length(past, s_new);
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kRopeWarps * 32, kRopeBlocksPerSm)
@@ -61,18 +81,22 @@ __global__ void __launch_bounds__(kRopeWarps * 32, kRopeBlocksPerSm)
   const int i0 = (sub % kPartner) * 8;  // index within the half of this lane's 8 elements
   const int slots = p.Hq + 2 * p.Hkv;
 
+  // Safe only because total_lens never overlaps past_lens here (the host
+  // then leaves total_lens to rope_lengths_kernel, launched after this one).
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.B; i += gridDim.x * blockDim.x)
-    if (p.total_lens != nullptr) p.total_lens[i] = __ldg(p.past_lens + i) + p.S_new;
+    if (p.total_lens != nullptr) p.total_lens[i] = rope_total_length(__ldg(p.past_lens + i), p.S_new);
 
   for (int bt = blockIdx.x; bt < p.tokens; bt += gridDim.x) {  // block-uniform
     const int b = bt / p.S_new;
     const int t = bt - b * p.S_new;
     const int past = __ldg(p.past_lens + b);
-    const int pos = past + t;
-    if (past < 0 || pos >= p.cap || pos >= p.max_pos) {
+    // pos = past + t must lie in [0, min(cap, max_pos)); tested without
+    // forming past + t, which overflows for a corrupt past near INT_MAX
+    if (past < 0 || past > p.cap - 1 - t || past > p.max_pos - 1 - t) {
       if (threadIdx.x == 0) atomicOr(&g_error_word, kErrSeqlen);
       continue;
     }
+    const int pos = past + t;
     const float4* cr = reinterpret_cast<const float4*>(p.cos_t + static_cast<int64_t>(pos) * kHalf + i0);
     const float4* sr = reinterpret_cast<const float4*>(p.sin_t + static_cast<int64_t>(pos) * kHalf + i0);
     const float4 c0 = __ldg(cr), c1 = __ldg(cr + 1), s0 = __ldg(sr), s1 = __ldg(sr + 1);

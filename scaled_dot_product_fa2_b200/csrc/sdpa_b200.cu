@@ -253,13 +253,18 @@ constexpr double kSatCtas = 75.0;     // CTAs that saturate HBM (per-CTA rate ~ 
 constexpr double kWaveFixed = 330.0;  // per-wave start-up and drain, in tile-times of the whole device
 
 double decode_grid_cost(int64_t ctas, int t, int64_t slots) {
-  double cost = 0.0;
-  for (int64_t left = ctas; left > 0; left -= slots) {
-    const double n = static_cast<double>(std::min(left, slots));
-    cost += t * std::max(n, kSatCtas) + kWaveFixed;
-  }
+  const int64_t full = ctas / slots, rem = ctas - full * slots;
+  double cost = static_cast<double>(full) * (t * std::max(static_cast<double>(slots), kSatCtas) + kWaveFixed);
+  if (rem > 0) cost += t * std::max(static_cast<double>(rem), kSatCtas) + kWaveFixed;
   return cost;
 }
+
+// Each split count s is tried once, with the fewest tiles per split that give
+// exactly s splits, in increasing order (ties go to more splits: more CTAs in
+// flight).  Counts above kMaxAutoSplitsPerSlot * slots never win under the
+// model (one full wave already keeps every slot busy; more only adds waves),
+// so the search stops there and stays short for caches of any length.
+constexpr int kMaxAutoSplitsPerSlot = 4;
 
 int decode_tiles_per_split(int64_t pairs, int total_tiles, int sms, int requested_splits) {
   if (total_tiles <= 0) return 1;
@@ -268,13 +273,14 @@ int decode_tiles_per_split(int64_t pairs, int total_tiles, int sms, int requeste
     return (total_tiles + s - 1) / s;
   }
   const int64_t slots = static_cast<int64_t>(sms) * kDecCtasPerSm;
+  const int64_t max_s = std::min<int64_t>(total_tiles, kMaxAutoSplitsPerSlot * slots);
   int best_t = total_tiles;
   double best = 1e300;
-  for (int t = total_tiles; t >= 1; --t) {
-    const int64_t splits = (total_tiles + t - 1) / t;
-    if (t > 1 && (total_tiles + t - 2) / (t - 1) == splits) continue;  // same split count, fewer tiles each
-    const double cost = decode_grid_cost(pairs * splits, t, slots);
-    if (cost <= best * (1.0 + 1e-9)) {  // ties go to more splits (more CTAs in flight)
+  for (int64_t s = 1; s <= max_s; ++s) {
+    const int t = static_cast<int>((total_tiles + s - 1) / s);
+    if ((total_tiles + t - 1) / t != s) continue;  // s splits are not reachable exactly
+    const double cost = decode_grid_cost(pairs * s, t, slots);
+    if (cost <= best * (1.0 + 1e-9)) {
       best = cost;
       best_t = t;
     }
@@ -288,6 +294,7 @@ bool decode_shape(int B, int Hq, int Hkv, int Sq, int Sk, int d, int num_splits,
   if (Sq > kMaxSeq || Sk > kMaxSeq || num_splits < 0) return false;
   const int group = Hq / Hkv;
   const int64_t rows = static_cast<int64_t>(group) * Sq;
+  if (rows > INT_MAX) return false;  // the kernel indexes a KV head's query rows in int
   const int rg = static_cast<int>((rows + kDecRows - 1) / kDecRows);
   const int total_tiles = (Sk + kDecKeys - 1) / kDecKeys;
   const int64_t pairs = static_cast<int64_t>(B) * Hkv * rg;
@@ -374,15 +381,32 @@ attn_status_t launch_bwd(const BwdParams& prm, int dev, cudaStream_t st) {
 
 // Blocks for the rotary/append kernel: one per token, at most one resident
 // wave (kRopeBlocksPerSm per SM); the blocks stride over the remaining tokens.
+// When total_lens overlaps past_lens (lengths advanced in place) the append
+// kernel leaves it alone and a second kernel, ordered after it on the stream,
+// writes it.
 template <int D>
 attn_status_t launch_rope(const RopeParams& prm, int sms, cudaStream_t st) {
   const int64_t wave = static_cast<int64_t>(sms) * kRopeBlocksPerSm;
   const int grid = static_cast<int>(std::min<int64_t>(std::max(prm.tokens, 1), wave));
-  rope_append_kernel<D><<<grid, kRopeWarps * 32, 0, st>>>(prm);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  const uintptr_t pl = reinterpret_cast<uintptr_t>(prm.past_lens), tl = reinterpret_cast<uintptr_t>(prm.total_lens);
+  const uintptr_t n = static_cast<uintptr_t>(prm.B) * sizeof(int);
+  const bool overlap = prm.total_lens != nullptr && pl < tl + n && tl < pl + n;
+  RopeParams main = prm;
+  if (overlap) main.total_lens = nullptr;
+  rope_append_kernel<D><<<grid, kRopeWarps * 32, 0, st>>>(main);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (overlap) {
+    rope_lengths_kernel<<<static_cast<unsigned>((prm.B + 255) / 256), 256, 0, st>>>(prm.past_lens, prm.total_lens,
+                                                                                    prm.B, prm.S_new);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
 }
 
 }  // namespace
+
+// Whether the current device can run the library's kernels (ATTN_ERR_ARCH if not).
+attn_status_t current_device_status() { return current_device(nullptr, nullptr); }
 }  // namespace sdpa
 
 using namespace sdpa;
@@ -491,7 +515,8 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int d,
 
 static attn_status_t decode_impl(const void* q, const void* k_cache, const void* v_cache, const attn_extras_t* ex,
                                  void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale,
-                                 int causal, int num_splits, void* workspace, size_t workspace_bytes, void* stream) {
+                                 int causal, int num_splits, void* workspace, size_t workspace_bytes, void* stream,
+                                 bool withhold_loads = false) {
   attn_status_t s = check_common(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
   if (s != ATTN_OK) return s;
   if ((s = check_extras(ex, B, Hq, false)) != ATTN_OK) return s;
@@ -548,6 +573,7 @@ static attn_status_t decode_impl(const void* q, const void* k_cache, const void*
   prm.scale = sc;
   prm.scale_log2 = sc * 1.4426950408889634f;
   prm.inv_scale = 1.f / sc;
+  prm.withhold_loads = withhold_loads ? 1 : 0;
   const int64_t grid = static_cast<int64_t>(B) * Hkv * ns * rg;
   if (grid > INT_MAX || (rows + 3) / 4 > INT_MAX) return ATTN_ERR_SHAPE;
   if (d == 128) return launch_decode<128>(prm, static_cast<int>(grid), part_o, part_ml, o, lse, rows, dev, st);
@@ -582,6 +608,14 @@ attn_status_t attn_decode_splitkv_ex(const void* q, const void* k_cache, const v
                                      const attn_extras_t* extras, void* stream) {
   return decode_impl(q, k_cache, v_cache, extras, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal, num_splits,
                      workspace, workspace_bytes, stream);
+}
+
+attn_status_t attn_selftest_decode_wait_timeout(const void* q, const void* k_cache, const void* v_cache, void* o,
+                                                float* lse, int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (B <= 0 || Sq <= 0 || Sk <= 0) return ATTN_ERR_SHAPE;  // the kernel must have something to wait for
+  return decode_impl(q, k_cache, v_cache, nullptr, o, lse, B, Hq, Hkv, Sq, Sk, d, 0.f, ATTN_CAUSAL_BOTTOM_RIGHT, 0,
+                     workspace, workspace_bytes, stream, /*withhold_loads=*/true);
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int Sq) {
@@ -749,7 +783,10 @@ std::mutex g_static_scratch_mu;
 
 // Device address of the scratch array on the current device (looked up once per
 // device, with that device current).  Host code cannot use the symbol itself:
-// on the host it names a stand-in, not device memory.
+// on the host it names a stand-in, not device memory.  The cached address
+// assumes the device's primary context lives as long as the process; a caller
+// that resets the device (cudaDeviceReset) must not call this entry point
+// again in that process.
 attn_status_t static_scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= sdpa::kMaxDeviceSlots) return ATTN_ERR_CUDA;
@@ -770,6 +807,8 @@ extern "C" attn_status_t attn_decode_splitkv_static(const void* q, const void* k
   attn_status_t s = check_common(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
   if (s != ATTN_OK) return s;
   if (num_splits < 0) return ATTN_ERR_SHAPE;
+  // the device must be a B200 before its copy of the scratch is looked up
+  if (B > 0 && Sq > 0 && (s = sdpa::current_device_status()) != ATTN_OK) return s;
   if (B > 0 && Sq > 0 && Sk > 0) {
     const size_t need = attn_decode_workspace_size(B, Hq, Hkv, Sq, Sk, d, num_splits);
     if (need == 0) return ATTN_ERR_SHAPE;

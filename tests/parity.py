@@ -56,6 +56,29 @@ def oracle_rows(q, k, v, scale, causal, rows):
     return oracle.attn_rows(q.double().numpy(), k.double().numpy(), v.double().numpy(), scale, causal, rows)
 
 
+def nan_outputs(q, B, Hq, Sq):
+    """Output buffers pre-filled with NaN: a row the kernel never writes stays
+    NaN, so a skipped or mis-dealt work unit cannot pass as finite stale data."""
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full((B, Hq, Sq), float("nan"), dtype=torch.float32, device=q.device)
+    return o, lse
+
+
+def tile_rows(B, Hq, Sq, seed=0, tile=128):
+    """Flattened rows: one seeded random row inside every ``tile``-row query
+    tile of every (batch, head), plus each head's first and last row.  Each
+    work unit of the forward (a batch, a head, a pair of 128-row query tiles)
+    then has rows of both its tiles in the sample."""
+    rng = np.random.default_rng(seed)
+    n_t = (Sq + tile - 1) // tile
+    bh = np.repeat(np.arange(B * Hq, dtype=np.int64), n_t)
+    t = np.tile(np.arange(n_t, dtype=np.int64), B * Hq)
+    size = np.minimum(tile, Sq - t * tile)
+    i = t * tile + (rng.random(bh.shape[0]) * size).astype(np.int64)
+    edges = np.concatenate([np.arange(B * Hq, dtype=np.int64) * Sq, np.arange(B * Hq, dtype=np.int64) * Sq + Sq - 1])
+    return np.unique(np.concatenate([bh * Sq + i, edges]))
+
+
 def sample_rows(B, Hq, Sq, n_random=96, seed=0):
     """Flattened (b*Hq + h)*Sq + i rows: tile edges, the ragged end, random rows."""
     rng = np.random.default_rng(seed)

@@ -100,21 +100,27 @@ def test_fwd_varlen_out_of_range_lengths_are_clamped_and_reported(sdpa):
 
 def test_fwd_varlen_long_gqa_sampled_rows(sdpa):
     """GQA at long lengths (several 256-row units per batch, one much shorter
-    batch): every row of the short batch and sampled rows of the long one."""
+    batch), into NaN-filled outputs: every valid row must be written and every
+    padding row left alone; one oracle row from every 128-row query tile of
+    every head of both batches."""
     B, Hq, Hkv, S = 2, 32, 8, 4096
     lq, lk = [4096, 1500], [4096, 3000]
     q, k, v = parity.seeded(B, Hq, Hkv, S, S, 128, seed=84)
-    o, lse = run(sdpa, q, k, v, lq, lk, BR)
+    qd, kd, vd = parity.to_dev(q, k, v)
+    o, lse = parity.nan_outputs(qd, B, Hq, S)
+    sq = torch.tensor(lq, dtype=torch.int32, device="cuda")
+    sk = torch.tensor(lk, dtype=torch.int32, device="cuda")
+    sdpa.attn_fwd_varlen(qd, kd, vd, sq, sk, causal=BR, out=o, lse=lse)
     sdpa.check_device_error()
     o = o.float().cpu().numpy()
     lse = lse.cpu().numpy()
     scale = 1 / math.sqrt(128)
-    rows0 = parity.sample_rows(1, Hq, lq[0], n_random=64, seed=5)
-    o_ref, lse_ref = parity.oracle_rows(q[0:1], k[0:1], v[0:1], scale, BR, rows0)
-    parity.compare(o[0].reshape(-1, 128)[rows0], lse[0].reshape(-1)[rows0], o_ref, lse_ref, "long batch")
-    rows1 = parity.sample_rows(1, Hq, lq[1], n_random=64, seed=6)
-    o_ref, lse_ref = parity.oracle_rows(q[1:2, :, :lq[1]], k[1:2, :, :lk[1]], v[1:2, :, :lk[1]], scale, BR, rows1)
-    got_o = o[1, :, :lq[1]].reshape(-1, 128)[rows1]
-    got_l = lse[1, :, :lq[1]].reshape(-1)[rows1]
-    parity.compare(got_o, got_l, o_ref, lse_ref, "short batch")
-    assert not np.any(o[1, :, lq[1]:])
+    for b in range(B):
+        assert np.isfinite(o[b, :, :lq[b]]).all() and np.isfinite(lse[b, :, :lq[b]]).all(), f"batch {b} unwritten"
+        assert np.isnan(o[b, :, lq[b]:]).all() and np.isnan(lse[b, :, lq[b]:]).all(), f"batch {b} padding written"
+        rows = parity.tile_rows(1, Hq, lq[b], seed=5 + b)
+        o_ref, lse_ref = parity.oracle_rows(q[b:b + 1, :, :lq[b]], k[b:b + 1, :, :lk[b]], v[b:b + 1, :, :lk[b]],
+                                            scale, BR, rows)
+        got_o = o[b, :, :lq[b]].reshape(-1, 128)[rows]
+        got_l = lse[b, :, :lq[b]].reshape(-1)[rows]
+        parity.compare(got_o, got_l, o_ref, lse_ref, f"batch {b}")

@@ -188,6 +188,30 @@ def test_decode_split_policy_fills_one_wave(lib):
 
 
 
+def test_decode_split_policy_is_quick_for_any_cache_length(lib):
+    """The automatic split search is bounded: a cache of 2^30 keys (16M tiles)
+    with many (batch, kv head) pairs is sized in well under a second."""
+    import time
+    t0 = time.perf_counter()
+    for B, Hkv in [(1, 1), (64, 8), (1024, 64)]:
+        ns = lib.attn_decode_num_splits(B, Hkv * 4, Hkv, 1, 1 << 30, 128)
+        assert ns >= 1
+        assert lib.attn_decode_workspace_size(B, Hkv * 4, Hkv, 1, 1 << 30, 128, 0) > 0
+    assert time.perf_counter() - t0 < 1.0
+
+
+def test_decode_rejects_query_rows_per_kv_head_beyond_int(lib):
+    # group * Sq = 65536 * 32768 = 2^31 query rows share one KV head
+    assert lib.attn_decode_workspace_size(1, 1 << 16, 1, 1 << 15, 128, 128, 0) == 0
+    assert lib.attn_decode_num_splits(1, 1 << 16, 1, 1 << 15, 128, 128) == 0
+
+
+def test_selftest_timeout_entry_rejects_empty_problems_on_host(lib):
+    P = ctypes.c_void_p(16)
+    for B, Sq, Sk in [(0, 1, 1), (1, 0, 1), (1, 1, 0)]:
+        assert lib.attn_selftest_decode_wait_timeout(P, P, P, P, None, B, 4, 1, Sq, Sk, 128, P, 1 << 20, None) == 2
+
+
 def test_rope_append_rejects_bad_arguments_on_host(lib):
     def call(packed=P, cos=P, sin=P, max_pos=64, past=P, q=P, kc=P, vc=P, tot=P, B=2, S_new=3, Hq=4, Hkv=2,
              cap=64, d=128, layout=0):

@@ -1,9 +1,11 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
 
 Small shapes are compared element by element in full (several 128-row tiles,
-ragged tails, every causal mode, GQA, d = 64 and 128, edge cases); the
-full-size workloads are compared on sampled rows the oracle computes one by
-one, in the launch configuration the benchmark uses.
+ragged tails, every causal mode, GQA, d = 64 and 128, edge cases).  The
+full-size workloads run in the launch configuration the benchmark uses, into
+NaN-filled outputs (every row must be written): each is compared on one
+oracle row from every 128-row query tile, and two whole workloads (causal
+seq 2048, non-causal seq 4096) element by element.
 """
 import math
 
@@ -59,6 +61,8 @@ SMALL = [
     (1, 2, 2, 1, 1000, 128, BR),       # one query at the end of 1000 keys
     (3, 2, 2, 7, 129, 128, NONE),      # ragged both ways, tiny
     (1, 1, 1, 1024, 1024, 128, TL),    # 4 units, exercises LPT ordering
+    (4, 40, 8, 520, 520, 128, TL),     # 480 units > 148 CTAs: several dealing rounds, GQA group 5
+    (3, 32, 32, 300, 700, 64, BR),     # 192 units > 148 CTAs at d = 64 (8-slot ring)
 ]
 
 
@@ -126,24 +130,50 @@ def test_large_magnitude_inputs_stay_finite(sdpa):
     parity.compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, "large scores")
 
 
-# ------------------------------------------------------------- full-size workloads (sampled rows)
+# ------------------------------------------------------------- full-size workloads
 
 FULL = inputs.PREFILL_NONCAUSAL + inputs.PREFILL_CAUSAL + [inputs.GQA_LONG]
 
 
-@pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
-def test_prefill_full_size_sampled(sdpa, w):
+def run_full_size(sdpa, w):
+    """The workload in the benchmark's launch configuration, into NaN-filled outputs."""
     q, k, v = inputs.workload_inputs(w)
     qd, kd, vd = parity.to_dev(q, k, v)
-    o, lse = sdpa.attn_fwd(qd, kd, vd, causal=w.causal, scale=w.scale)
+    o, lse = parity.nan_outputs(qd, w.B, w.Hq, w.Sq)
+    sdpa.attn_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=o, lse=lse)
     sdpa.check_device_error()
-    rows = parity.sample_rows(w.B, w.Hq, w.Sq, seed=w.seed)
+    # every row of every work unit was written (the buffers started as NaN)
+    assert torch.isfinite(o).all(), f"{w.name}: rows of O left unwritten"
+    assert torch.isfinite(lse).all(), f"{w.name}: LSE entries left unwritten"
+    return (q, k, v), o, lse
+
+
+@pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
+def test_prefill_full_size_every_tile_sampled(sdpa, w):
+    """One oracle row inside every 128-row query tile of every head, so every
+    work unit of the persistent schedule (all rounds of its snake dealing) is
+    checked against the oracle, not only a random handful."""
+    (q, k, v), o, lse = run_full_size(sdpa, w)
+    rows = parity.tile_rows(w.B, w.Hq, w.Sq, seed=w.seed)
     o_ref, lse_ref = parity.oracle_rows(q, k, v, w.eff_scale, w.causal, rows)
-    o_g = o.reshape(-1, w.d)[torch.from_numpy(rows).cuda()].float().cpu().numpy()
-    l_g = lse.reshape(-1)[torch.from_numpy(rows).cuda()].cpu().numpy()
+    idx = torch.from_numpy(rows).cuda()
+    o_g = o.reshape(-1, w.d)[idx].float().cpu().numpy()
+    l_g = lse.reshape(-1)[idx].cpu().numpy()
     parity.compare(o_g, l_g, o_ref, lse_ref, w.name)
-    # properties that hold at any size: finite everywhere
-    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+
+
+WHOLE = [inputs.BY_NAME["prefill_causal_s2048"], inputs.BY_NAME["prefill_noncausal_s4096"]]
+
+
+@pytest.mark.parametrize("w", WHOLE, ids=lambda w: w.name)
+def test_prefill_whole_workload_element_by_element(sdpa, w):
+    """Every element of a whole benchmark workload against the oracle: 1024
+    work units over the 148-CTA persistent grid, so the multi-round snake
+    dealing and the ring and barrier phases that run on across units are
+    checked on every row."""
+    (q, k, v), o, lse = run_full_size(sdpa, w)
+    o_ref, lse_ref = parity.oracle_full(q, k, v, w.eff_scale, w.causal)
+    parity.compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, w.name)
 
 
 # ------------------------------------------------------------- decode

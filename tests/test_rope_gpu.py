@@ -137,6 +137,53 @@ def test_rope_append_out_of_range_positions_are_skipped_and_reported(sdpa):
     assert torch.equal(kc_new[0, :, :cap - 2], kc[0, :, :cap - 2])
 
 
+def test_rope_append_lengths_advanced_in_place(sdpa):
+    """total_lens may be past_lens itself (the decode loop's in-place update):
+    every token must still be placed at its OLD length + t, across many blocks."""
+    B, S_new, Hq, Hkv, d, cap = 8, 40, 8, 2, 128, 160
+    packed, kc, vc, past_lens = inputs.make_rope_inputs(B, S_new, Hq, Hkv, d, cap, 7500)
+    cos, sin = inputs.rope_tables(cap, d)
+    kc_d, vc_d = kc.cuda(), vc.cuda()
+    lens_d = past_lens.cuda()
+    q_d, tot = sdpa.attn_rope_append(packed.cuda(), cos.cuda(), sin.cuda(), lens_d, kc_d, vc_d, Hq, Hkv,
+                                     total_lens=lens_d)
+    sdpa.check_device_error()
+    assert tot.data_ptr() == lens_d.data_ptr()
+    q_ref, k_ref, v_ref, tot_ref = oracle.rope_append(packed.double().numpy(), cos.double().numpy(),
+                                                      sin.double().numpy(), past_lens.numpy(),
+                                                      kc.double().numpy(), vc.double().numpy(), Hq, Hkv)
+    assert np.array_equal(lens_d.cpu().numpy(), tot_ref), "lengths advanced in place"
+    assert_close(q_d.cpu().double().numpy(), q_ref,
+                 rot_tolerance(packed, Hq, Hkv, d, slice(0, Hq)).transpose(0, 2, 1, 3), "q")
+    k_extra = rot_tolerance(packed, Hq, Hkv, d, slice(Hq, Hq + Hkv)).transpose(0, 2, 1, 3)
+    kc_new, vc_new = kc_d.cpu(), vc_d.cpu()
+    for b, p in enumerate(past_lens.tolist()):
+        sl = slice(p, p + S_new)
+        assert_close(kc_new[b, :, sl].double().numpy(), k_ref[b, :, sl], k_extra[b], f"k rows of batch {b}")
+        assert torch.equal(vc_new[b, :, sl], torch.from_numpy(v_ref[b, :, sl]).bfloat16()), f"v rows of batch {b}"
+
+
+def test_rope_append_past_length_near_int_max_is_skipped(sdpa):
+    """A corrupt past length near INT_MAX must not wrap into a negative
+    position: its tokens are skipped and reported, its cache rows untouched,
+    and its total length saturates at INT_MAX."""
+    B, S_new, Hq, Hkv, d, cap = 2, 3, 4, 2, 128, 16
+    big = 2 ** 31 - 2
+    packed, kc, vc, past_lens, cos, sin, q, kc_new, vc_new, tot = run_case(sdpa, B, S_new, Hq, Hkv, d, cap, 7600,
+                                                                           past=[big, 4])
+    with pytest.raises(_lib.AttnError) as e:
+        sdpa.check_device_error()
+    assert e.value.status == 13
+    sdpa.check_device_error()
+    assert tot.tolist() == [2 ** 31 - 1, 7]
+    assert not q[0].any(), "q rows of the skipped batch were written"
+    assert torch.equal(kc_new[0], kc[0]) and torch.equal(vc_new[0], vc[0]), "cache of the skipped batch changed"
+    q_ref, k_ref, _, _ = oracle.rope_append(packed[1:].double().numpy(), cos.double().numpy(), sin.double().numpy(),
+                                            np.array([4]), kc[1:].double().numpy(), vc[1:].double().numpy(), Hq, Hkv)
+    assert_close(q[1:].double().numpy(), q_ref,
+                 rot_tolerance(packed[1:], Hq, Hkv, d, slice(0, Hq)).transpose(0, 2, 1, 3), "q of batch 1")
+
+
 def test_rope_append_empty_inputs(sdpa):
     dev = "cuda"
     Hq, Hkv, d, cap = 4, 2, 64, 8
