@@ -33,6 +33,8 @@ import torch  # noqa: E402
 from scaled_dot_product_fa2_b200 import inputs  # noqa: E402
 
 HEADLINE = inputs.PREFILL_NONCAUSAL
+WORKLOAD_NAME = ("prefill non-causal d=128 H=16 seq {512,1024,2048,4096} B=16384/seq "
+                 "(one call per shape per step)")
 METRIC = "attn fwd TFLOP/s (bf16, d=128) and decode KV GB/s, as fraction of B200 roofline"
 L2_FLUSH_BYTES = 256 << 20
 # After each flush a short device-side spin keeps the GPU busy while the host
@@ -229,10 +231,42 @@ class CpuOracleSample:
             self.per_row = dt / n
         n = int(min(self.total_rows, max(self.threads, target_s / max(self.per_row, 1e-9))))
         rows, dt = self._run(n)
+        self.per_row = dt / n
         tflops = self._flops(rows) / dt / 1e12
         desc = (f"{n} random query rows of {self.w.name} (of {self.total_rows}), fp64 oracle on "
                 f"{self.threads} threads, {dt:.1f} s")
         return tflops, self.threads, desc, dt
+
+
+def oracle_per_config(target_s: float = 1.5):
+    """The oracle as it stands on every configuration: the tiny and decode
+    workloads in full, each prefill shape and the GQA workload on a seeded
+    random row sample whose measured per-row time is scaled to the full row
+    count (labelled "extrapolated")."""
+    import oracle
+    threads = os.cpu_count() or 1
+    out = {}
+    for w in [inputs.TINY] + list(inputs.DECODE):
+        q, k, v = inputs.workload_inputs(w)
+        qd, kd, vd = q.double().numpy(), k.double().numpy(), v.double().numpy()
+        t0 = time.perf_counter()
+        oracle.attn_fwd(qd, kd, vd, w.eff_scale, w.causal, nthreads=threads)
+        dt = time.perf_counter() - t0
+        rate = (w.flops() / dt / 1e12) if not w.decode else None
+        entry = {"full_s": round(dt, 4), "how": "measured on the whole workload", "threads": threads}
+        if w.decode:
+            entry["gbs"] = round(w.decode_bytes() / dt / 1e9, 3)
+        else:
+            entry["tflops"] = round(rate, 6)
+        out[w.name] = entry
+    for w in list(inputs.PREFILL_NONCAUSAL) + list(inputs.PREFILL_CAUSAL) + [inputs.GQA_LONG]:
+        sampler = CpuOracleSample(w)
+        tf, cores, desc, dt = sampler.sample(target_s=target_s)
+        full_s = sampler.per_row * sampler.total_rows
+        out[w.name] = {"tflops": round(tf, 6), "full_s": round(full_s, 2), "threads": cores,
+                       "how": f"extrapolated from {desc}"}
+        del sampler
+    return out
 
 
 # ------------------------------------------------------------------ GPU timing
@@ -501,8 +535,10 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tf, cores, desc, _ = CpuOracleSample(HEADLINE[-1]).sample(target_s=12.0)
-        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+        cpu = sweep_oracle_sample(target_s=8.0)
+        if not args.no_breakdown:
+            for name, entry in oracle_per_config().items():
+                breakdown.setdefault(name, {})["oracle"] = entry
 
     if rank == 0:
         line = {
@@ -511,8 +547,7 @@ def main():
             "wall_ms_per_step": round(wall * 1e3 / args.steps, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded randn N(0,1), rounded to bf16)",
-            "config": {"workload": "prefill non-causal d=128 H=16 seq {512,1024,2048,4096} B=16384/seq "
-                                   "(one call per shape per step)",
+            "config": {"workload": WORKLOAD_NAME,
                        "global_batch_tokens": 16384 * 4 * world, "seq_len": [w.Sq for w in HEADLINE],
                        "heads": 16, "head_dim": 128, "causal": False, "parallelism": f"replicas x{world}",
                        "l2": "flushed (256 MiB write) before every call",
@@ -533,6 +568,11 @@ def main():
 
 def measure_breakdown(flush, peak_tf, hbm_gbs, rank, reps: int = 10):
     out = {}
+    # the tiny causal workload (B=1, H=2, S=128, d=64): a launch-latency figure
+    s = GpuPrefill(inputs.TINY, rank)
+    ms = statistics.median(timed_calls([s.run], flush, reps, 3)[0])
+    out[inputs.TINY.name] = {"ms": round(ms, 4), "tflops": round(inputs.TINY.flops() / ms / 1e9, 3)}
+    del s
     for w in inputs.PREFILL_CAUSAL + [inputs.GQA_LONG]:
         s = GpuPrefill(w, rank)
         ms = statistics.median(timed_calls([s.run], flush, reps, 3)[0])
@@ -654,27 +694,57 @@ def run_profile_case(args):
     print(f"profile case {w.name}: {args.profile_calls} calls ok", flush=True)
 
 
+def sweep_oracle_sample(target_s: float):
+    """The oracle on a bounded sample of the headline workload itself: seeded
+    random query rows of every shape of the sweep, about target_s seconds in
+    all, split over the shapes in proportion to their FLOPs; TFLOP/s = the
+    sampled rows' algorithmic FLOPs / the time taken."""
+    total = sum(w.flops() for w in HEADLINE)
+    fl = dt = 0.0
+    nrows = []
+    cores = os.cpu_count() or 1
+    for w in HEADLINE:
+        sampler = CpuOracleSample(w)
+        t_share = target_s * w.flops() / total
+        if sampler.per_row is None:
+            n = min(sampler.total_rows, 8 * sampler.threads)
+            _, d0 = sampler._run(n)
+            sampler.per_row = d0 / n
+        n = int(min(sampler.total_rows, max(sampler.threads, t_share / max(sampler.per_row, 1e-9))))
+        rows, d = sampler._run(n)
+        fl += sampler._flops(rows)
+        dt += d
+        nrows.append(f"{n} of {w.name}")
+        cores = sampler.threads
+        del sampler
+    desc = (f"seeded random query rows of every shape of the sweep ({', '.join(nrows)}), fp64 oracle on "
+            f"{cores} threads, {dt:.1f} s")
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,
+            "seconds": round(dt, 2)}
+
+
 def run_reference(args, world, rank):
-    """The reference arm: the fp64 oracle as it stands, on the host cores,
-    on a bounded sample of the headline workload (rank 0 only)."""
+    """The reference arm: the fp64 oracle as it stands, on the host cores, on
+    a bounded sample of the same workload as this benchmark's own arm (every
+    shape of the non-causal sweep), rank 0 only."""
     if rank != 0:
         return
-    w = HEADLINE[-1]
-    sampler = CpuOracleSample(w)
     vals = []
+    per_step = max(1.0, 60.0 / max(1, args.warmup + args.steps))
     for i in range(args.warmup + args.steps):
-        tf, cores, desc, dt = sampler.sample(target_s=max(1.0, 60.0 / max(1, args.warmup + args.steps)))
+        c = sweep_oracle_sample(target_s=per_step)
         if i >= args.warmup:
-            vals.append((tf, dt))
-    tf = statistics.median(v for v, _ in vals)
+            vals.append(c)
+    tf = statistics.median(c["value"] for c in vals)
+    last = vals[-1]
     line = {"impl": "reference", "metric": METRIC, "value": round(tf, 6), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(1e3 * statistics.median(dt for _, dt in vals), 3),
+            "ms_per_step": round(1e3 * statistics.median(c["seconds"] for c in vals), 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded randn N(0,1), rounded to bf16)",
-            "config": {"workload": f"{w.name}: row sample of the prefill non-causal d=128 H=16 workload"},
-            "cpu_baseline": {"value": round(tf, 6), "unit": "TFLOP/s", "cores": os.cpu_count() or 1,
-                             "kind": "oracle", "sample": desc},
+            "config": {"workload": WORKLOAD_NAME + " (each step a seeded row sample of it)"},
+            "cpu_baseline": {"value": round(tf, 6), "unit": "TFLOP/s", "cores": last["cores"],
+                             "kind": "oracle", "sample": last["sample"]},
             "e2e": {"value": round(tf, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
