@@ -9,12 +9,19 @@
 // block) (same notes, improvement 2: sequence-length parallelism).
 //
 // B200 mapping (this file's own design, not the pages'):
-//   * Persistent grid: one CTA per SM walks a static list of work units
-//     (batch*head, pair of 128-row query tiles).  For causal masks the list
-//     holds the heaviest units (the last query tiles of each head) first and
-//     is dealt to the CTAs in snake order, round by round, which balances the
-//     per-SM work like longest-processing-time-first scheduling.  One unit's
-//     epilogue overlaps the next unit's loads and first MMAs.
+//   * Work units (batch*head, pair of 128-row query tiles) in a list that, for
+//     causal masks, holds the heaviest units (the last query tiles of each
+//     head) first.  One CTA fits on an SM.  Fixed lengths: a persistent grid
+//     of one CTA per SM deals the list round by round in snake order, which
+//     balances units of known cost like longest-processing-time-first.
+//     Per-batch lengths (units whose cost is only known on the device, many
+//     of them empty): the grid has one CTA per unit, and each running CTA,
+//     when it has issued the loads of its unit, takes the next unit whose CTA
+//     has not started by cancelling that CTA's launch (cluster launch
+//     control), so the SMs pull units from the list as they free up.  Either
+//     way one thread (the K/V producer) announces the CTA's units to the
+//     other roles through a small ring in shared memory.  One unit's epilogue
+//     overlaps the next unit's loads and first MMAs.
 //   * One CTA = two query tiles sharing every K/V tile it loads; 12 warps:
 //       warps 0-3  softmax group 0 (one thread per row of query tile 0)
 //       warps 4-7  softmax group 1 (query tile 1)
@@ -78,6 +85,7 @@ struct PrefillParams {
   int num_units;      // ceil(Sq / 256): work units per (batch, head)
   int total_units;    // B * Hq * num_units
   int lpt;            // 1: heaviest units first (causal)
+  int dynamic;        // 1: grid of one CTA per unit, units taken over at run time; 0: persistent snake deal
   float scale;        // softmax scale on q.k
   float scale_log2;   // scale * log2(e)
 };
@@ -100,6 +108,7 @@ constexpr int kCtrlRegsBias = 56;
 static_assert(256 * kSoftmaxRegsBias + 128 * kCtrlRegsBias == kPrefillThreads * kLaunchRegs,
               "register split must equal the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest P kept unrescaled
+constexpr int kUnitRing = 4;  // units announced ahead by the scheduling thread
 
 template <int D, int NS>
 struct PrefillCfg {
@@ -107,8 +116,12 @@ struct PrefillCfg {
   static constexpr int kBlocks = D / 64;               // 64-column swizzle blocks per tile
   static constexpr int kBlockBytes = kBlockM * 128;    // 16 KB per swizzle block
   // q_full[2] q_empty[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2] o_full[2] turn[2] drain
-  static constexpr int kNumBars = 4 + 2 * NS + 2 + 2 + 2 + 2 + 1;
-  static constexpr int kSmemBytes = (2 + NS) * kTileBytes + kNumBars * 8 + 16 + 1024;
+  // unit_full[kUnitRing] unit_empty[kUnitRing] clc
+  static constexpr int kNumBars = 4 + 2 * NS + 2 + 2 + 2 + 2 + 1 + 2 * kUnitRing + 1;
+  // after the barriers, 16-byte aligned: the cancel answer (16 bytes), the unit
+  // ring (kUnitRing ints), the TMEM base and the abort flag
+  static constexpr int kMiscOffset = (kNumBars * 8 + 15) / 16 * 16;
+  static constexpr int kSmemBytes = (2 + NS) * kTileBytes + kMiscOffset + 16 + 4 * kUnitRing + 8 + 1024;
 };
 
 // Number of 128-key tiles the query tile starting at row0 must visit, for a
@@ -124,8 +137,9 @@ __device__ __forceinline__ int kv_tiles_for(int causal, int Lq, int Lk, int coff
   return last_key / kBlockN + 1;
 }
 
-// The r-th work unit of CTA c in a grid of G CTAs: round r deals list entries
-// [r*G, r*G + G) in snake order (forward in even rounds, backward in odd).
+// The r-th work unit of CTA c in a persistent grid of G CTAs: round r deals
+// list entries [r*G, r*G + G) in snake order (forward in even rounds,
+// backward in odd).
 __device__ __forceinline__ int unit_index(int r, int c, int G) { return r * G + ((r & 1) ? (G - 1 - c) : c); }
 
 // Work-list entry -> (batch*head, pair index v of query tiles 2v, 2v+1).
@@ -243,14 +257,30 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
   auto o_full = [&](int t) { return bar0 + 8u * (8 + 2 * NS + t); };    // a unit's last P.V done
   auto turn = [&](int t) { return bar0 + 8u * (10 + 2 * NS + t); };     // tile t may issue
   const uint32_t drain = bar0 + 8u * (12 + 2 * NS);                     // every MMA done
+  auto unit_full = [&](int k) { return bar0 + 8u * (13 + 2 * NS + k); };              // ring entry k written
+  auto unit_empty = [&](int k) { return bar0 + 8u * (13 + 2 * NS + kUnitRing + k); }; // ring entry k read
+  const uint32_t clc_bar = bar0 + 8u * (13 + 2 * NS + 2 * kUnitRing);                 // cancel answer landed
   uint8_t* bar_ptr = smem + 2 * Cfg::kTileBytes + NS * Cfg::kTileBytes;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * Cfg::kNumBars);
+  uint8_t* misc = bar_ptr + Cfg::kMiscOffset;
+  const uint32_t clc_resp = smem_u32(misc);
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(misc + 16);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 16 + 4 * kUnitRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // The r-th unit of this CTA: wait for ring entry r, read it, release it.
+  // -1 ends the sequence.  The caller's whole warp (or its lone thread) calls
+  // it; one arrival per warp.
+  auto next_unit = [&](int r, bool& ok) -> int {
+    const int k = r % kUnitRing;
+    ok = ok && mbar_wait(unit_full(k), (r / kUnitRing) & 1, abort_flag);
+    if (!ok) return -1;
+    const int idx = unit_ring[k];
+    __syncwarp(__activemask());
+    if ((threadIdx.x & 31) == 0 || __activemask() == 1u) mbar_arrive(unit_empty(k));
+    return idx;
+  };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int cta = static_cast<int>(blockIdx.x);
-  const int G = static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
@@ -266,6 +296,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
       mbar_init(kv_empty(s), 2);  // released by both MMA threads
     }
     mbar_init(drain, 2);  // one commit per MMA thread
+    for (int k = 0; k < kUnitRing; ++k) {
+      mbar_init(unit_full(k), 1);
+      mbar_init(unit_empty(k), 2 + 8);  // both MMA threads and the eight softmax warps
+    }
+    mbar_init(clc_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -293,6 +328,24 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
         int it = 0;  // K/V tiles issued so far (ring position)
         int ui = 0;  // units started so far
         bool ok = true;
+        // This thread also schedules: it announces the CTA's units in the
+        // unit ring -- the persistent grid's snake deal, or (dynamic) its own
+        // unit first, then each one it takes over from a CTA that has not
+        // started -- and -1 when there is none left.
+        int clc_asked = 0;      // cancel requests issued (clc_bar phase)
+        bool clc_pending = false;
+        auto announce = [&](int r, int v) -> bool {
+          const int k = r % kUnitRing;
+          if (r >= kUnitRing && !mbar_wait(unit_empty(k), ((r / kUnitRing) - 1) & 1, abort_flag)) return false;
+          unit_ring[k] = v;
+          mbar_arrive(unit_full(k));  // release: the entry is visible to whoever sees the phase
+          return true;
+        };
+        const int cta = static_cast<int>(blockIdx.x);
+        const int G = static_cast<int>(gridDim.x);
+        int idx = p.dynamic ? cta : unit_index(0, cta, G);
+        if (idx >= p.total_units) idx = -1;
+        ok = announce(0, idx);
         // Q_0 and Q_1 of unit u, each once the previous unit's last S MMA on
         // that buffer is done (a tile with no key tiles only completes the phase).
         auto load_q = [&](const Unit& u) -> bool {
@@ -310,9 +363,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
           return true;
         };
 #pragma unroll 1
-        for (int r = 0; ok; ++r) {
-          const int idx = unit_index(r, cta, G);
-          if (idx >= p.total_units) break;
+        for (int r = 0; ok && idx >= 0; ++r) {
           const Unit u = make_unit(p, idx);
           if (p.seqlens_q != nullptr || p.seqlens_k != nullptr) {
             const int b = u.bh / p.Hq;
@@ -340,7 +391,37 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
                           kv_full(slot));
           }
           ++ui;
+          if (!ok) break;
+          // The next unit: the snake deal's, or (dynamic) the first one in the
+          // list whose CTA has not started.
+          int next = -1;
+          if (!p.dynamic) {
+            next = unit_index(r + 1, cta, G);
+            if (next >= p.total_units) next = -1;
+          } else if (clc_asked >= 0) {
+            mbar_arrive_expect_tx(clc_bar, 16);
+            clc_try_cancel(clc_resp, clc_bar);
+            clc_pending = true;
+            if (!mbar_wait(clc_bar, clc_asked & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            clc_pending = false;
+            ++clc_asked;
+            next = clc_canceled_x(clc_resp);
+            if (next < 0 || next >= p.total_units) {
+              next = -1;
+              clc_asked = -1;  // never ask again after a refusal
+            }
+          }
+          if (!announce(r + 1, next)) {
+            ok = false;
+            break;
+          }
+          idx = next;
         }
+        // An answer still on its way must land before the CTA may exit.
+        if (clc_pending) mbar_wait_drain(clc_bar, clc_asked & 1);
         // Copies still in flight must land before the CTA may exit.
         if (ui > 0) {
           mbar_wait_drain(q_full(0), (ui - 1) & 1);
@@ -376,8 +457,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
         bool ok = true;
 #pragma unroll 1
         for (int r = 0; ok; ++r) {
-          const int idx = unit_index(r, cta, G);
-          if (idx >= p.total_units) break;
+          const int idx = next_unit(r, ok);
+          if (idx < 0) break;
           const Unit u = make_unit(p, idx);
           const int nt = t ? u.n1 : u.n0;  // n0 <= n1: tile 1's rows come later
           if (!mbar_wait(q_full(t), ui & 1, abort_flag)) break;
@@ -457,8 +538,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
     bool ok = true;
 #pragma unroll 1
     for (int r = 0; ok; ++r) {
-      const int idx = unit_index(r, cta, G);
-      if (idx >= p.total_units) break;
+      const int idx = next_unit(r, ok);  // warp-uniform
+      if (idx < 0) break;
       const Unit u = make_unit(p, idx);
       const int row0 = u.row0_0 + t * kBlockM;
       const int row = row0 + r_in_tile;

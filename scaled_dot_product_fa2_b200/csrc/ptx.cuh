@@ -120,6 +120,34 @@ __device__ __forceinline__ void tma_load_4d(uint32_t smem_dst, const CUtensorMap
       : "memory");
 }
 
+// ------------------------------------------------------- cluster launch control
+// Ask the hardware to cancel the launch of a CTA of this grid that has not
+// started yet, so that this CTA can do its work instead.  The 16-byte answer
+// lands at `resp` (16-byte aligned shared memory) and completes 16 bytes of
+// transaction on `bar`.  After one failed request a CTA must not ask again.
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(resp),
+      "r"(bar)
+      : "memory");
+}
+
+// Decode an answer of clc_try_cancel: the x index of the canceled CTA, or -1
+// if nothing was canceled (no CTA of the grid was still waiting to start).
+__device__ __forceinline__ int clc_canceled_x(uint32_t resp) {
+  uint32_t canceled, x;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b128 q;\n\t"
+      "ld.shared.b128 q, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, q;\n\t}"
+      : "=r"(canceled), "=r"(x)
+      : "r"(resp)
+      : "memory");
+  return canceled ? static_cast<int>(x) : -1;
+}
+
 // ------------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t smem_slot, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_slot), "r"(ncols)

@@ -465,8 +465,11 @@ static attn_status_t fwd_impl(const void* q, const void* k, const void* v, const
   const int64_t units = static_cast<int64_t>(B) * Hq * prm.num_units;
   if (units > INT_MAX / 2) return ATTN_ERR_SHAPE;
   prm.total_units = static_cast<int>(units);
-  // Persistent grid: one CTA per SM (the kernel's shared memory allows one).
-  const int64_t grid = std::min<int64_t>(units, sms);
+  // Fixed lengths: persistent grid, one CTA per SM (the kernel's shared memory
+  // allows one).  Per-batch lengths: one CTA per unit, running CTAs take over
+  // the units of CTAs that have not started (see prefill.cuh).
+  prm.dynamic = (prm.seqlens_q != nullptr || prm.seqlens_k != nullptr) ? 1 : 0;
+  const int64_t grid = prm.dynamic ? units : std::min<int64_t>(units, sms);
   if (d == 128) {
     return has_bias ? launch_prefill<128, kStagesD128, true>(prm, static_cast<int>(grid), dev, st)
                     : launch_prefill<128, kStagesD128, false>(prm, static_cast<int>(grid), dev, st);

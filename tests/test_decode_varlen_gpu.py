@@ -116,3 +116,24 @@ def test_varlen_decode_workload_sampled_rows(sdpa, w):
     sdpa.check_device_error()
     o_ref, lse_ref = per_batch_oracle(q, k, v, lens, w.eff_scale, w.causal)
     parity.compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, w.name + " varlen")
+
+
+
+SKEWED = [
+    # lengths, Hq, Hkv, Sq, capacity
+    ([8192] + [0] * 7, 32, 8, 4, 8192),                       # one full batch, the rest empty
+    ([5, 4000, 0, 8191, 64, 65, 1, 3000] * 5, 8, 2, 1, 8192),  # 40 batches of every kind of length
+    ([300, 1, 299], 64, 2, 1, 300),                           # 32 query rows per kv head: two row groups
+    ([2] * 200, 4, 4, 1, 64),                                 # 800 (batch, kv head) pairs, more than one wave
+]
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,Sq,cap", SKEWED, ids=["one_full", "b40", "two_row_groups", "many_pairs"])
+def test_varlen_skewed_length_mixes(sdpa, lens, Hq, Hkv, Sq, cap):
+    """Extreme mixes of per-batch lengths against the per-batch oracle."""
+    B = len(lens)
+    q, k, v = parity.seeded(B, Hq, Hkv, Sq, cap, 128, seed=740 + B + Hq)
+    o, lse = run_varlen(sdpa, q, k, v, lens, BR)
+    sdpa.check_device_error()
+    o_ref, lse_ref = per_batch_oracle(q, k, v, lens, 1 / math.sqrt(128), BR)
+    parity.compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, f"lens {lens[:4]}")
