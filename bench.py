@@ -683,6 +683,9 @@ def run_profile_case(args):
         # the backward pass of a prefill workload, e.g. bwd_prefill_noncausal_s4096
         w = inputs.BY_NAME[args.profile[len("bwd_"):]]
         runner = GpuBackward(w, 0)
+    elif args.profile == inputs.PREFILL_VARLEN.name:
+        w = inputs.PREFILL_VARLEN
+        runner = GpuPrefillVarlen(w, 0)
     else:
         w = inputs.BY_NAME[args.profile]
         runner = GpuDecode(w, 0) if w.decode else GpuPrefill(w, 0)
