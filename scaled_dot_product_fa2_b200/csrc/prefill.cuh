@@ -60,6 +60,7 @@
 #pragma once
 #include <climits>
 
+#include "fastdiv.h"
 #include "ptx.cuh"
 
 namespace sdpa {
@@ -88,6 +89,9 @@ struct PrefillParams {
   int dynamic;        // 1: grid of one CTA per unit, units taken over at run time; 0: persistent snake deal
   float scale;        // softmax scale on q.k
   float scale_log2;   // scale * log2(e)
+  // the same divisions by launch constants as multiply-highs (no division
+  // instruction sequence at a unit boundary): by B*Hq, Hq, group, num_units
+  FastDiv div_bh, div_hq, div_group, div_units;
 };
 
 constexpr int kBlockM = 128;  // query rows per tile
@@ -146,11 +150,12 @@ __device__ __forceinline__ int unit_index(int r, int c, int G) { return r * G + 
 __device__ __forceinline__ void unit_coords(const PrefillParams& p, int idx, int& bh, int& v) {
   const int BH = p.B * p.Hq;
   if (p.lpt) {
-    v = p.num_units - 1 - idx / BH;
-    bh = idx % BH;
+    const int r = static_cast<int>(fastdiv(static_cast<uint32_t>(idx), p.div_bh));
+    v = p.num_units - 1 - r;
+    bh = idx - r * BH;
   } else {
-    v = idx % p.num_units;
-    bh = idx / p.num_units;
+    bh = static_cast<int>(fastdiv(static_cast<uint32_t>(idx), p.div_units));
+    v = idx - bh * p.num_units;
   }
 }
 
@@ -168,11 +173,11 @@ __device__ __forceinline__ Unit make_unit(const PrefillParams& p, int idx) {
   Unit u;
   int v;
   unit_coords(p, idx, u.bh, v);
-  const int b = u.bh / p.Hq;
+  const int b = static_cast<int>(fastdiv(static_cast<uint32_t>(u.bh), p.div_hq));
   const int hq = u.bh - b * p.Hq;
   u.b = b;
   u.hq = hq;
-  u.hkv = hq / p.group;
+  u.hkv = static_cast<int>(fastdiv(static_cast<uint32_t>(hq), p.div_group));
   u.row0_0 = v * 2 * kBlockM;
   u.Lq = batch_length(p.seqlens_q, b, p.Sq);
   u.Lk = batch_length(p.seqlens_k, b, p.Sk);
@@ -226,7 +231,7 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint6
 // pointer kept live across the softmax step would cost registers it needs.
 template <int C0>
 __device__ __forceinline__ void load_bias_chunks(const PrefillParams& p, int bh, int row, int k0, uint4 (&bz)[16]) {
-  const int b = bh / p.Hq;
+  const int b = static_cast<int>(fastdiv(static_cast<uint32_t>(bh), p.div_hq));
   const uint16_t* brow = p.bias + b * p.bias_sb + (bh - b * p.Hq) * p.bias_sh + static_cast<int64_t>(row) * p.Sk;
 #pragma unroll
   for (int c8 = C0; c8 < C0 + 8; ++c8) {
@@ -366,7 +371,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
         for (int r = 0; ok && idx >= 0; ++r) {
           const Unit u = make_unit(p, idx);
           if (p.seqlens_q != nullptr || p.seqlens_k != nullptr) {
-            const int b = u.bh / p.Hq;
+            const int b = static_cast<int>(fastdiv(static_cast<uint32_t>(u.bh), p.div_hq));
             const bool bad_q = p.seqlens_q != nullptr && __ldg(p.seqlens_q + b) != u.Lq;
             const bool bad_k = p.seqlens_k != nullptr && __ldg(p.seqlens_k + b) != u.Lk;
             if (bad_q || bad_k) atomicOr(&g_error_word, kErrSeqlen);
@@ -665,11 +670,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
       if (!ok) break;
 
       // ---- epilogue: O / l -> bf16 -> global.  Each thread normalises its own
-      // row; then, per 64 columns, an 8 x 8 transpose of 16-byte chunks inside
-      // each group of 8 lanes (xor shuffles) lets every store instruction
-      // write four whole 128-byte row segments instead of 32 scattered
-      // 16-byte pieces (which made the epilogue ~3.5k cycles on the tile's
-      // critical path).
+      // row; then, per 64 columns, a transpose of row chunks between the lanes
+      // of a small group (xor shuffles) makes every store instruction write
+      // whole 128-byte row segments instead of 32 scattered pieces.  The
+      // epilogue sits on the tile's path from one unit to the next, so its
+      // cost counts once per unit (about 10 % of a causal seq-2048 unit).
       if (row0 < u.Lq) {
         if (n > 0) {
           if (!mbar_wait(o_full(t), ou & 1, abort_flag)) ok = false;
@@ -684,6 +689,62 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
         const int g = lane & 7;
         const int group_row0 = row0 + wq * 32 + (lane & ~7);  // first row of this lane's group of 8
         uint16_t* const o_head = p.o + u.b * p.o_sb + u.hq * p.o_sh;
+        if ((reinterpret_cast<uintptr_t>(p.o) & 31u) == 0u) {
+          // 32-byte aligned rows.  Per 64 columns (128 bytes of a row = four
+          // 32-byte chunks), a 4 x 4 transpose of chunks inside each group of
+          // 4 lanes (xor shuffles), after which every 32-byte store of the warp
+          // writes eight whole 128-byte row segments.
+          const int g4 = lane & 3;
+          const int grp_row0 = row0 + wq * 32 + (lane & ~3);
+          const float2 il2 = make_float2(inv_l, inv_l);
+#pragma unroll 1
+          for (int h = 0; h < D / 64; ++h) {
+            uint32_t o0[32], o1[32];
+            if (have_o) {
+              tmem_ld32(tO + h * 64, o0);
+              tmem_ld32(tO + h * 64 + 32, o1);
+              tmem_wait_ld();
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o0[e] = o1[e] = 0u;
+            }
+            uint32_t w[4][8];  // chunk c = columns 64 h + 16 c .. + 15 of this lane's row
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint32_t* f = (c < 2) ? &o0[c * 16] : &o1[(c - 2) * 16];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float2 x = __fmul2_rn(make_float2(__uint_as_float(f[2 * e]), __uint_as_float(f[2 * e + 1])), il2);
+                w[c][e] = pack_bf16x2(x.x, x.y);
+              }
+            }
+#pragma unroll
+            for (int sft = 2; sft > 0; sft >>= 1) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                if (i & sft) continue;
+                const int jj = i | sft;
+                const bool upper = (g4 & sft) != 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const uint32_t x = upper ? w[i][e] : w[jj][e];
+                  const uint32_t y = __shfl_xor_sync(0xffffffffu, x, sft);
+                  if (upper) {
+                    w[i][e] = y;
+                  } else {
+                    w[jj][e] = y;
+                  }
+                }
+              }
+            }
+            // lane g4 now holds chunk g4 of rows grp_row0 + 0..3 in w[0..3]
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int rr = grp_row0 + i;
+              if (rr < u.Lq) st_global_v8(o_head + static_cast<int64_t>(rr) * p.o_sr + h * 64 + g4 * 16, w[i]);
+            }
+          }
+        } else
 #pragma unroll 1
         for (int h = 0; h < D / 64; ++h) {
           uint32_t o0[32], o1[32];

@@ -465,6 +465,10 @@ static attn_status_t fwd_impl(const void* q, const void* k, const void* v, const
   const int64_t units = static_cast<int64_t>(B) * Hq * prm.num_units;
   if (units > INT_MAX / 2) return ATTN_ERR_SHAPE;
   prm.total_units = static_cast<int>(units);
+  prm.div_bh = make_fastdiv(static_cast<uint32_t>(std::max(B * Hq, 1)));
+  prm.div_hq = make_fastdiv(static_cast<uint32_t>(std::max(Hq, 1)));
+  prm.div_group = make_fastdiv(static_cast<uint32_t>(std::max(prm.group, 1)));
+  prm.div_units = make_fastdiv(static_cast<uint32_t>(std::max(prm.num_units, 1)));
   // Fixed lengths: persistent grid, one CTA per SM (the kernel's shared memory
   // allows one).  Per-batch lengths: one CTA per unit, running CTAs take over
   // the units of CTAs that have not started (see prefill.cuh).

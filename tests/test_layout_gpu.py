@@ -73,3 +73,25 @@ def test_decode_bshd_query_matches_default_layout(sdpa, Sq):
         assert torch.equal(o1.transpose(1, 2), o2) and torch.equal(l1, l2)
     o_ref, lse_ref = parity.oracle_full(q, k, v, 1 / math.sqrt(d), BR)
     parity.compare(o1.transpose(1, 2).float().cpu().numpy(), l1.cpu().numpy(), o_ref, lse_ref, "bshd decode")
+
+
+@pytest.mark.parametrize("d,causal,layout", [(128, TL, 0), (64, NONE, 0), (128, BR, 1)])
+def test_forward_output_aligned_to_16_bytes_only(sdpa, d, causal, layout):
+    """An output buffer 16 bytes past a 32-byte boundary takes the epilogue's
+    16-byte store path; it must write the same bits as a 32-byte aligned one."""
+    from scaled_dot_product_fa2_b200 import ops
+    B, Hq, Hkv, Sq, Sk = 2, 4, 2, 300, 517
+    q, k, v = parity.seeded(B, Hq, Hkv, Sq, Sk, d, seed=1300 + d + causal)
+    qd, kd, vd = parity.to_dev(q, k, v)
+    lay = ops.LAYOUT_BSHD if layout else ops.LAYOUT_BHSD
+    if layout:
+        qd, kd, vd = bshd(qd), bshd(kd), bshd(vd)
+    o_ref, l_ref = sdpa.attn_fwd(qd, kd, vd, causal=causal, layout=lay)
+    flat = torch.full((qd.numel() + 64,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    start = (32 - flat.data_ptr() % 32) // 2 + 8  # 16 bytes past a 32-byte boundary
+    o_off = flat[start:start + qd.numel()].view(qd.shape)
+    assert o_off.data_ptr() % 32 == 16
+    o2, l2 = sdpa.attn_fwd(qd, kd, vd, causal=causal, layout=lay, out=o_off)
+    sdpa.check_device_error()
+    assert torch.equal(o2, o_ref) and torch.equal(l2, l_ref)
+    assert torch.isnan(flat[:start]).all() and torch.isnan(flat[start + qd.numel():]).all()
