@@ -28,7 +28,7 @@
 //       warp  8    MMA issuer for query tile 0 (one elected thread) + TMEM owner
 //       warp  9    TMA producer (one elected thread)
 //       warp 10    MMA issuer for query tile 1
-//       warp 11    idle
+//       warp 11    bias tile loader (bias variant), else idle
 //     Each query tile has its own MMA-issuing thread.  On B200 any
 //     shared-memory access (an mbarrier wait included) by a thread that has
 //     just issued tcgen05.mma stalls it for 120-210 cycles, while only about
@@ -54,6 +54,11 @@
 //     than the MMA itself.
 //   * Rescaling of O is skipped unless the running max grows by more than
 //     2^8 in the exp2 domain (exact: the final O/l and LSE use the same m).
+//   * Bias variant: warp 11 stages each (query tile, key tile) bias tile by TMA
+//     into one 32 KB buffer that the two tiles' softmax steps use in turn
+//     (tile 0 step j, tile 1 step j, tile 0 step j + 1, ...); the softmax
+//     reads its row's 16-byte chunks at their 128-byte-swizzle positions.  The
+//     buffer costs one K/V slot (4 instead of 5 at d = 128).
 //   * The epilogue writes O/l from registers straight to global memory, so a
 //     tile's Q buffer is free as soon as its last S MMA is done and the next
 //     unit's Q can load while this unit finishes.
@@ -71,6 +76,9 @@ struct PrefillParams {
   CUtensorMap tm_q;
   CUtensorMap tm_k;
   CUtensorMap tm_v;
+  // 4-D map (Sk, Sq, bias_h, bias_b) over the additive bias, box {64, 128, 1, 1},
+  // 128-byte swizzle, zero fill outside (bias variant only)
+  CUtensorMap tm_bias;
   uint16_t* o;       // bf16 bits; element (b, h, i, c) at b*o_sb + h*o_sh + i*o_sr + c
   int64_t o_sb, o_sh, o_sr;
   float* lse;        // [B*Hq*Sq] or nullptr
@@ -78,6 +86,7 @@ struct PrefillParams {
   const int* seqlens_k;  // [B] valid keys of each batch (device), or nullptr: all Sk
   const uint16_t* bias;  // bf16 additive bias [bias_b][bias_h][Sq][Sk] (Sk % 8 == 0), or nullptr
   int64_t bias_sb, bias_sh;  // its batch and head strides in elements (0 where it broadcasts)
+  int bias_per_b, bias_per_h;  // 1 where the bias has its own plane per batch / per query head
   float inv_scale;       // 1 / scale: the bias enters the raw scores as bias / scale
   int B, Hq, Hkv, Sq, Sk;
   int group;          // Hq / Hkv
@@ -101,6 +110,7 @@ constexpr int kPrefillThreads = 384;
 constexpr int kMmaWarp = 8;    // query tile 0; also allocates and frees TMEM
 constexpr int kLoadWarp = 9;
 constexpr int kMmaWarp1 = 10;  // query tile 1
+constexpr int kBiasWarp = 11;  // bias variant: loads the bias tiles
 constexpr int kLaunchRegs = 168;  // 3 warps per SM sub-partition: 3*32*168 <= 16384
 constexpr int kSoftmaxRegs = 216;
 constexpr int kCtrlRegs = 72;
@@ -114,18 +124,23 @@ static_assert(256 * kSoftmaxRegsBias + 128 * kCtrlRegsBias == kPrefillThreads * 
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest P kept unrescaled
 constexpr int kUnitRing = 4;  // units announced ahead by the scheduling thread
 
-template <int D, int NS>
+template <int D, int NS, bool BIAS = false>
 struct PrefillCfg {
   static constexpr int kTileBytes = kBlockM * D * 2;  // one Q, K or V tile (bf16)
+  // bias variant: one 128-row x 128-key bf16 bias tile, staged by TMA, which
+  // the two query tiles' softmax steps use in turn
+  static constexpr int kBiasTileBytes = BIAS ? kBlockM * kBlockN * 2 : 0;
   static constexpr int kBlocks = D / 64;               // 64-column swizzle blocks per tile
   static constexpr int kBlockBytes = kBlockM * 128;    // 16 KB per swizzle block
   // q_full[2] q_empty[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2] o_full[2] turn[2] drain
-  // unit_full[kUnitRing] unit_empty[kUnitRing] clc
-  static constexpr int kNumBars = 4 + 2 * NS + 2 + 2 + 2 + 2 + 1 + 2 * kUnitRing + 1;
+  // unit_full[kUnitRing] unit_empty[kUnitRing] clc bias_full[2] bias_empty[2]
+  static constexpr int kNumBars = 4 + 2 * NS + 2 + 2 + 2 + 2 + 1 + 2 * kUnitRing + 1 + 4;
   // after the barriers, 16-byte aligned: the cancel answer (16 bytes), the unit
   // ring (kUnitRing ints), the TMEM base and the abort flag
   static constexpr int kMiscOffset = (kNumBars * 8 + 15) / 16 * 16;
-  static constexpr int kSmemBytes = (2 + NS) * kTileBytes + kMiscOffset + 16 + 4 * kUnitRing + 8 + 1024;
+  static constexpr int kSmemBytes =
+      (2 + NS) * kTileBytes + kBiasTileBytes + kMiscOffset + 16 + 4 * kUnitRing + 8 + 1024;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
 };
 
 // Number of 128-key tiles the query tile starting at row0 must visit, for a
@@ -225,34 +240,20 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint6
   }
 }
 
-// Bias of one query row for keys k0 + 8*c .. k0 + 8*c + 7, c in [C0, C0 + 8),
-// as bf16 pairs (row or keys out of the bias give zeros: those scores are
-// masked or never written).  The row's address is recomputed at each call: a
-// pointer kept live across the softmax step would cost registers it needs.
-template <int C0>
-__device__ __forceinline__ void load_bias_chunks(const PrefillParams& p, int bh, int row, int k0, uint4 (&bz)[16]) {
-  const int b = static_cast<int>(fastdiv(static_cast<uint32_t>(bh), p.div_hq));
-  const uint16_t* brow = p.bias + b * p.bias_sb + (bh - b * p.Hq) * p.bias_sh + static_cast<int64_t>(row) * p.Sk;
-#pragma unroll
-  for (int c8 = C0; c8 < C0 + 8; ++c8) {
-    const int key = k0 + c8 * 8;
-    bz[c8] = (row < p.Sq && key < p.Sk) ? __ldg(reinterpret_cast<const uint4*>(brow + key))
-                                         : make_uint4(0u, 0u, 0u, 0u);
-  }
-}
-
 // BIAS: add the additive attention bias to the scores (a separate
 // instantiation, so the common path carries none of its loads).
 template <int D, int NS, bool BIAS>
 __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
-  using Cfg = PrefillCfg<D, NS>;
+  using Cfg = PrefillCfg<D, NS, BIAS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // Shared-memory map (32-bit shared addresses):
-  //   sQ   2 query tiles, sKV NS key/value slots, then the barriers.
+  //   sQ   2 query tiles, sKV NS key/value slots, (bias variant) sBias one bias
+  //   tile, then the barriers.
   const uint32_t sQ = smem_u32(smem);
   const uint32_t sKV = sQ + 2 * Cfg::kTileBytes;
-  const uint32_t bar0 = sKV + NS * Cfg::kTileBytes;
+  const uint32_t sBias = sKV + NS * Cfg::kTileBytes;
+  const uint32_t bar0 = sBias + Cfg::kBiasTileBytes;
   auto q_full = [&](int t) { return bar0 + 8u * t; };                   // Q_t landed
   auto q_empty = [&](int t) { return bar0 + 8u * (2 + t); };            // Q_t's last S MMA done
   auto kv_full = [&](int s) { return bar0 + 8u * (4 + s); };            // slot filled
@@ -265,7 +266,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
   auto unit_full = [&](int k) { return bar0 + 8u * (13 + 2 * NS + k); };              // ring entry k written
   auto unit_empty = [&](int k) { return bar0 + 8u * (13 + 2 * NS + kUnitRing + k); }; // ring entry k read
   const uint32_t clc_bar = bar0 + 8u * (13 + 2 * NS + 2 * kUnitRing);                 // cancel answer landed
-  uint8_t* bar_ptr = smem + 2 * Cfg::kTileBytes + NS * Cfg::kTileBytes;
+  auto bias_full = [&](int t) { return bar0 + 8u * (14 + 2 * NS + 2 * kUnitRing + t); };   // bias tile t landed
+  auto bias_empty = [&](int t) { return bar0 + 8u * (16 + 2 * NS + 2 * kUnitRing + t); };  // bias tile t read
+  uint8_t* bar_ptr = smem + 2 * Cfg::kTileBytes + NS * Cfg::kTileBytes + Cfg::kBiasTileBytes;
   uint8_t* misc = bar_ptr + Cfg::kMiscOffset;
   const uint32_t clc_resp = smem_u32(misc);
   volatile int* unit_ring = reinterpret_cast<volatile int*>(misc + 16);
@@ -295,6 +298,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
       mbar_init(p_full(t), 4);  // one arrive per softmax warp
       mbar_init(turn(t), 1);
       mbar_init(o_full(t), 1);
+      mbar_init(bias_full(t), 1);
+      mbar_init(bias_empty(t), 4);  // one arrive per softmax warp of tile t
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(kv_full(s), 1);
@@ -303,7 +308,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
     mbar_init(drain, 2);  // one commit per MMA thread
     for (int k = 0; k < kUnitRing; ++k) {
       mbar_init(unit_full(k), 1);
-      mbar_init(unit_empty(k), 2 + 8);  // both MMA threads and the eight softmax warps
+      mbar_init(unit_empty(k), 2 + 8 + (BIAS ? 1 : 0));  // MMA threads, softmax warps (bias loader)
     }
     mbar_init(clc_bar, 1);
     *abort_flag = 0;
@@ -435,6 +440,49 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
         for (int i = max(0, it - NS); i < it; ++i) mbar_wait_drain(kv_full(i % NS), (i / NS) & 1);
       }
       __syncwarp();
+    } else if (BIAS && warp == kBiasWarp) {
+      // ---------------------------------------------------- bias loader
+      // The bias tile of (query tile t, key tile j) -- 128 rows x 128 keys,
+      // two 64-key boxes -- into the bias buffer, in the order the softmax
+      // steps use them (tile 0 step j, tile 1 step j, tile 0 step j + 1, ...),
+      // each once the previous tile's softmax warps have read theirs; rows
+      // and keys outside the bias read as zero (those scores are masked or
+      // never written).
+      if (lane == 0) {
+        tma_prefetch_desc(&p.tm_bias);
+        int loaded[2] = {0, 0};  // bias tiles loaded for each query tile
+        int prev_t = -1;         // query tile of the previous load
+        bool ok = true;
+#pragma unroll 1
+        for (int r = 0; ok; ++r) {
+          const int idx = next_unit(r, ok);
+          if (idx < 0) break;
+          const Unit u = make_unit(p, idx);
+          const int hb = p.bias_per_h ? u.hq : 0;
+          const int bb = p.bias_per_b ? u.b : 0;
+#pragma unroll 1
+          for (int j = 0; ok && j < u.n_max; ++j) {
+            for (int t = 0; t < 2 && ok; ++t) {
+              if (j >= (t ? u.n1 : u.n0)) continue;
+              if (prev_t >= 0 && !mbar_wait(bias_empty(prev_t), (loaded[prev_t] - 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              mbar_arrive_expect_tx(bias_full(t), Cfg::kBiasTileBytes);
+              const uint32_t dst = sBias;
+              for (int blk = 0; blk < 2; ++blk)
+                tma_load_4d(dst + blk * (kBlockM * 128), &p.tm_bias, j * kBlockN + blk * 64, u.row0_0 + t * kBlockM,
+                            hb, bb, bias_full(t));
+              ++loaded[t];
+              prev_t = t;
+            }
+          }
+        }
+        // the last copy must land before the CTA may exit (the earlier ones
+        // were all read)
+        if (prev_t >= 0) mbar_wait_drain(bias_full(prev_t), (loaded[prev_t] - 1) & 1);
+      }
+      __syncwarp();
     } else if (warp == kMmaWarp || warp == kMmaWarp1) {
       // ---------------------------------------------- MMA issuer of tile t
       // Segment k of tile t in a unit is O_t += P_t(k-1) V_{k-1} (k >= 1)
@@ -555,11 +603,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
 
 #pragma unroll 1
       for (int j = 0; j < n; ++j, ++sj) {
-        // The bias of this key tile's first 64 keys is fetched before the wait
-        // for S, so its latency overlaps the wait; the second 64 right after
-        // (keys past Sk read nothing: they are masked).
-        uint4 bz[BIAS ? 16 : 1];
-        if constexpr (BIAS) load_bias_chunks<0>(p, u.bh, row, j * kBlockN, bz);
         if (!mbar_wait(s_full(t), sj & 1, abort_flag)) {
           ok = false;
           break;
@@ -571,10 +614,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
           for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[q * 32]));
           tmem_wait_ld();
         } else {
-          // S in two 64-column halves, each given its bias as soon as it lands
-          // (fewer registers live at once than all of S plus all of the bias).
+          // S in two 64-column halves, each given its bias from the staged
+          // bias tile: this thread's row, 16-byte chunks of 8 keys at the
+          // 128-byte swizzle's position (chunk c of row r at c ^ (r mod 8)).
           const float2 is2 = make_float2(p.inv_scale, p.inv_scale);
-          load_bias_chunks<8>(p, u.bh, row, j * kBlockN, bz);
+          if (!mbar_wait(bias_full(t), sj & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t brow = sBias + static_cast<uint32_t>(r_in_tile) * 128u;
+          const uint32_t bsw = static_cast<uint32_t>(r_in_tile & 7);
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             tmem_ld32(tS + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[half * 64]));
@@ -582,7 +631,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
             tmem_wait_ld();
 #pragma unroll
             for (int c8 = half * 8; c8 < half * 8 + 8; ++c8) {
-              const uint32_t w[4] = {bz[c8].x, bz[c8].y, bz[c8].z, bz[c8].w};
+              const uint4 bz = ld_shared_u4(brow + half * (kBlockM * 128) + ((static_cast<uint32_t>(c8 & 7) ^ bsw) << 4));
+              const uint32_t w[4] = {bz.x, bz.y, bz.z, bz.w};
 #pragma unroll
               for (int u2 = 0; u2 < 4; ++u2) {
                 const int e = c8 * 8 + u2 * 2;
@@ -594,6 +644,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const __gri
               }
             }
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bias_empty(t));  // this warp's rows of the bias tile are read
         }
         const int k0 = j * kBlockN;
         const bool need_mask = (k0 + kBlockN > u.Lk) || (p.causal && k0 + kBlockN - 1 > row0 + u.coff);

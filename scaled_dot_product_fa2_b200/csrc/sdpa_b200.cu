@@ -172,9 +172,31 @@ bool make_map4(CUtensorMap* map, const void* base, int layout, int B, int H, int
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D bf16 map (Sk, Sq, Hb, Bb) over an additive bias [Bb][Hb][Sq][Sk] (Hb, Bb
+// are 1 where it broadcasts); box {64 keys, 128 rows, 1, 1}, 128-byte
+// swizzle, zero fill outside.  Sk % 8 == 0 and a 16-byte aligned base
+// (checked by the caller) make the row stride a multiple of 16 bytes.
+bool make_bias_map(CUtensorMap* map, const void* base, int Bb, int Hb, int Sq, int Sk) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(Sk), static_cast<cuuint64_t>(Sq), static_cast<cuuint64_t>(Hb),
+                              static_cast<cuuint64_t>(Bb)};
+  const cuuint64_t row = static_cast<cuuint64_t>(Sk) * 2;
+  const cuuint64_t strides[3] = {row, row * static_cast<cuuint64_t>(Sq),
+                                 row * static_cast<cuuint64_t>(Sq) * static_cast<cuuint64_t>(Hb)};
+  const cuuint32_t box[4] = {64, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------ kernels' config
 constexpr int kStagesD128 = 5;
 constexpr int kStagesD64 = 8;
+// The bias variant stages a 32 KB bias tile in shared memory, which leaves
+// room for 4 K/V slots at d = 128.
+constexpr int kStagesD128Bias = 4;
 constexpr int kDecStages = 3;   // 3 x 32 KB ring: two decode CTAs fit on one SM
 constexpr int kDecCtasPerSm = 2;
 
@@ -221,7 +243,7 @@ template <int D, int NS, bool BIAS>
 attn_status_t launch_prefill(const PrefillParams& prm, int grid, int dev, cudaStream_t st) {
   static bool smem_done[kMaxDevices] = {};
   static std::mutex mu;
-  using Cfg = PrefillCfg<D, NS>;
+  using Cfg = PrefillCfg<D, NS, BIAS>;
   {
     std::lock_guard<std::mutex> lock(mu);
     if (!smem_done[dev]) {
@@ -448,6 +470,9 @@ static attn_status_t fwd_impl(const void* q, const void* k, const void* v, const
   if (has_bias) {
     prm.bias = static_cast<const uint16_t*>(ex->bias);
     bias_strides(ex, Sq, Sk, &prm.bias_sb, &prm.bias_sh);
+    prm.bias_per_b = ex->bias_b == 1 ? 0 : 1;
+    prm.bias_per_h = ex->bias_h == 1 ? 0 : 1;
+    if (!make_bias_map(&prm.tm_bias, ex->bias, ex->bias_b, ex->bias_h, Sq, Sk)) return ATTN_ERR_CUDA;
   }
   prm.B = B;
   prm.Hq = Hq;
@@ -475,7 +500,7 @@ static attn_status_t fwd_impl(const void* q, const void* k, const void* v, const
   prm.dynamic = (prm.seqlens_q != nullptr || prm.seqlens_k != nullptr) ? 1 : 0;
   const int64_t grid = prm.dynamic ? units : std::min<int64_t>(units, sms);
   if (d == 128) {
-    return has_bias ? launch_prefill<128, kStagesD128, true>(prm, static_cast<int>(grid), dev, st)
+    return has_bias ? launch_prefill<128, kStagesD128Bias, true>(prm, static_cast<int>(grid), dev, st)
                     : launch_prefill<128, kStagesD128, false>(prm, static_cast<int>(grid), dev, st);
   }
   return has_bias ? launch_prefill<64, kStagesD64, true>(prm, static_cast<int>(grid), dev, st)

@@ -69,6 +69,30 @@ def test_forward_bias_d64_gqa_and_zero_bias_equals_no_bias(sdpa):
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("causal", [NONE, TL])
+def test_forward_bias_many_units_sampled_rows(sdpa, causal):
+    """More work units than SMs (2 x 16 heads x 8 units of 256 rows), so every
+    CTA takes several units and the bias tiles stream through their staging
+    buffer across unit boundaries (and, causal, past the shorter tile's last
+    step); outputs NaN-prefilled; one oracle row from every 128-row tile."""
+    import oracle as oracle_mod
+    B, Hq, Hkv, S, d = 2, 16, 16, 2048, 128
+    q, k, v = parity.seeded(B, Hq, Hkv, S, S, d, seed=930 + causal)
+    bias = make_bias((1, Hq), S, S, seed=931 + causal)
+    qd, kd, vd = parity.to_dev(q, k, v)
+    o, lse = parity.nan_outputs(qd, B, Hq, S)
+    sdpa.attn_fwd(qd, kd, vd, causal=causal, bias=bias.cuda(), out=o, lse=lse)
+    sdpa.check_device_error()
+    # written rows are finite (a row whose every key is masked has O = 0, LSE = -inf)
+    assert not torch.isnan(o).any() and not torch.isnan(lse).any(), "a row was never written"
+    rows = parity.tile_rows(B, Hq, S, seed=932 + causal)
+    o_ref, lse_ref = oracle_mod.attn_rows(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                          1 / math.sqrt(d), causal, rows, bias=bias.double().numpy())
+    got_o = o.float().cpu().numpy().reshape(-1, d)[rows]
+    got_l = lse.cpu().numpy().reshape(-1)[rows]
+    parity.compare(got_o, got_l, o_ref, lse_ref, f"fwd bias many units causal={causal}")
+
+
 @pytest.mark.parametrize("dims", ["11", "BH"])
 @pytest.mark.parametrize("Sq,causal", [(1, BR), (4, BR), (3, NONE)])
 def test_decode_bias_matches_oracle(sdpa, dims, Sq, causal):
