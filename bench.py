@@ -320,6 +320,21 @@ class GpuPrefillVarlen(GpuPrefill):
         return sum(2.0 * self.w.Hq * L * L * self.w.d for L in self.lens)
 
 
+class GpuPrefillBias(GpuPrefill):
+    """A prefill workload with an additive bias shared by all heads and batches
+    ([1, 1, S, S] bf16, seeded N(0, 1))."""
+
+    def __init__(self, w, rank: int):
+        super().__init__(w, rank)
+        g = torch.Generator().manual_seed(w.seed + 99)
+        self.bias = torch.randn((1, 1, w.Sq, w.Sk), generator=g).bfloat16().cuda()
+
+    def run(self):
+        import scaled_dot_product_fa2_b200 as sdpa
+        sdpa.attn_fwd(self.q, self.k, self.v, causal=self.w.causal, scale=self.w.scale, out=self.o, lse=self.lse,
+                      bias=self.bias)
+
+
 class GpuDecode:
     def __init__(self, w, rank: int, copies: int = 3):
         import scaled_dot_product_fa2_b200 as sdpa
@@ -583,19 +598,12 @@ def measure_breakdown(flush, peak_tf, hbm_gbs, rank, reps: int = 10):
     # and batches ([1, 1, S, S] bf16, 8 MiB: it stays in L2, so this measures
     # the bias path's compute cost)
     wb = inputs.BY_NAME["prefill_noncausal_s2048"]
-    sb = GpuPrefill(wb, rank)
-    gb = torch.Generator().manual_seed(wb.seed + 99)
-    bias = torch.randn((1, 1, wb.Sq, wb.Sk), generator=gb).bfloat16().cuda()
-
-    def run_bias(sb=sb, bias=bias):
-        import scaled_dot_product_fa2_b200 as sdpa
-        sdpa.attn_fwd(sb.q, sb.k, sb.v, causal=wb.causal, scale=wb.scale, out=sb.o, lse=sb.lse, bias=bias)
-
-    ms = statistics.median(timed_calls([run_bias], flush, reps, 3)[0])
+    sb = GpuPrefillBias(wb, rank)
+    ms = statistics.median(timed_calls([sb.run], flush, reps, 3)[0])
     tf = wb.flops() / ms / 1e9
     out[wb.name + "_bias"] = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac": round(tf / peak_tf, 4),
                               "bias": "[1, 1, S, S] bf16"}
-    del sb, bias
+    del sb
 
     sv = GpuPrefillVarlen(inputs.PREFILL_VARLEN, rank)
     ms = statistics.median(timed_calls([sv.run], flush, reps, 3)[0])
@@ -686,6 +694,10 @@ def run_profile_case(args):
     elif args.profile == inputs.PREFILL_VARLEN.name:
         w = inputs.PREFILL_VARLEN
         runner = GpuPrefillVarlen(w, 0)
+    elif args.profile.endswith("_bias"):
+        # a prefill workload with the [1, 1, S, S] bias, e.g. prefill_noncausal_s2048_bias
+        w = inputs.BY_NAME[args.profile[:-len("_bias")]]
+        runner = GpuPrefillBias(w, 0)
     else:
         w = inputs.BY_NAME[args.profile]
         runner = GpuDecode(w, 0) if w.decode else GpuPrefill(w, 0)

@@ -22,13 +22,17 @@
 //                     key row, one for each half of the 128 query columns;
 //                     each half's bf16 results overwrite that half's first
 //                     32 columns of S^T and dP^T), then dV += P^T dO and
-//                     dK += dS^T Q with P^T, dS^T read from TMEM.
+//                     dK += dS^T Q with P^T, dS^T read from TMEM.  The next
+//                     tile's S^T is issued right after dV and its dP^T after
+//                     dK, each with its own commit, so its P^T (the
+//                     exponentials) is under way while dK and dP^T run.
 //   bwd_dq_kernel     one CTA per 128-row query tile: Q and dO stay in shared
 //                     memory while the key tiles stream; S = Q K^T and
 //                     dP = dO V^T, dS by the compute warps into TMEM columns
 //                     of its own, dQ += dS K.  With dS apart from S, the next
-//                     tile's S and dP are issued before this tile's dS K, so
-//                     the compute warps wait for two matmuls a tile, not three.
+//                     tile's S and dP are issued before this tile's dS K, and
+//                     S and dP have commits of their own: the compute warps
+//                     take the exponentials of S while dP and dS K run.
 // Fully masked key tiles are skipped (causal).  TMEM holds every accumulator
 // (dK and dV for the whole query loop, dQ for the whole key loop).  Every
 // wait is bounded; a timeout sets the device error word and the kernel exits.
@@ -93,9 +97,9 @@ struct BwdCfg {
   static constexpr int kVecBytes = 128 * 4;         // 128 fp32 (L2 or D of one query tile)
   // smem: two resident tiles, then per stage two streamed tiles and two vectors
   static constexpr int kStageBytes = 2 * kTileBytes + 2 * kVecBytes;
-  // res_full, st_full[2], st_empty[2], s_full, p_full, done, ds_free (dQ only: the
-  // previous dS has been read)
-  static constexpr int kNumBars = 1 + 2 * kBwdStages + 4;
+  // res_full, st_full[2], st_empty[2], s_full, p_full, done, then dK/dV: dp_full;
+  // dQ: ds_free (the previous dS has been read), dp_full
+  static constexpr int kNumBars = 1 + 2 * kBwdStages + 5;
   static constexpr int kSmemBytes = 2 * kTileBytes + kBwdStages * kStageBytes + kNumBars * 8 + 16 + 1024;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
   static constexpr uint32_t kTmemCols = 512;
@@ -135,27 +139,36 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __grid_constant__ B
   }
 }
 
-// P^T and dS^T for 32 query columns col0 .. col0+31 of one key row: sv, dp
-// hold S^T and dP^T, l2v / ddv the query tile's LSE*log2(e) and D; columns
-// before cmin do not see the key.  Results as bf16 pairs.
-__device__ __forceinline__ void dkdv_chunk(const uint32_t (&sv)[32], const uint32_t (&dp)[32], const float* l2v,
-                                           const float* ddv, int col0, int cmin, float c, uint32_t (&pk)[16],
-                                           uint32_t (&dk16)[16]) {
+// P^T and dS^T for 32 query columns col0 .. col0+31 of one key row, in two
+// passes, so that P^T can be computed as soon as S^T is in TMEM, before dP^T
+// is: P (fp32, kept for the second pass) and P^T as bf16 pairs from S^T
+// (sv) and the query tile's LSE*log2(e) (l2v); then dS^T from P, dP^T (dp)
+// and D (ddv).  Columns before cmin do not see the key.
+__device__ __forceinline__ void p_chunk(const uint32_t (&sv)[32], const float* l2v, int col0, int cmin, float c,
+                                        float (&pr)[32], uint32_t (&pk)[16]) {
 #pragma unroll
   for (int e = 0; e < 32; e += 4) {
     const float4 lv = *reinterpret_cast<const float4*>(l2v + col0 + e);
-    const float4 dv4 = *reinterpret_cast<const float4*>(ddv + col0 + e);
     const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
-    const float dq4[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
-    float pr[4], ds[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const float x = fmaf(__uint_as_float(sv[e + u]), c, -lq[u]);
-      pr[u] = (col0 + e + u >= cmin) ? ex2_approx(x) : 0.f;
-      ds[u] = pr[u] * (__uint_as_float(dp[e + u]) - dq4[u]);
+      pr[e + u] = (col0 + e + u >= cmin) ? ex2_approx(x) : 0.f;
     }
-    pk[e / 2] = pack_bf16x2(pr[0], pr[1]);
-    pk[e / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
+    pk[e / 2] = pack_bf16x2(pr[e], pr[e + 1]);
+    pk[e / 2 + 1] = pack_bf16x2(pr[e + 2], pr[e + 3]);
+  }
+}
+
+__device__ __forceinline__ void ds_chunk(const float (&pr)[32], const uint32_t (&dp)[32], const float* ddv, int col0,
+                                         uint32_t (&dk16)[16]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) {
+    const float4 dv4 = *reinterpret_cast<const float4*>(ddv + col0 + e);
+    const float dq4[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+    float ds[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) ds[u] = pr[e + u] * (__uint_as_float(dp[e + u]) - dq4[u]);
     dk16[e / 2] = pack_bf16x2(ds[0], ds[1]);
     dk16[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
   }
@@ -179,9 +192,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
   const uint32_t res_full = bar0;
   auto st_full = [&](int st) { return bar0 + 8u * (1 + st); };
   auto st_empty = [&](int st) { return bar0 + 8u * (1 + kBwdStages + st); };
-  const uint32_t s_full = bar0 + 8u * (1 + 2 * kBwdStages);
+  const uint32_t s_full = bar0 + 8u * (1 + 2 * kBwdStages);  // S^T of the current query tile done
   const uint32_t p_full = s_full + 8u;
   const uint32_t done = p_full + 8u;
+  const uint32_t dp_full = done + 8u;  // dP^T of the current query tile done
   uint8_t* bar_ptr = smem + 2 * Cfg::kTileBytes + kBwdStages * Cfg::kStageBytes;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * Cfg::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -207,6 +221,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     mbar_init(s_full, 1);
     mbar_init(p_full, kBwdComputeWarps);  // one arrive per compute warp
     mbar_init(done, 1);
+    mbar_init(dp_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -256,20 +271,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       const uint64_t dk_k = hi | sdesc_lo(sK, 16);  // K, K-major (A of S^T)
       const uint64_t dv_k = hi | sdesc_lo(sV, 16);  // V, K-major (A of dP^T)
       bool ok = mbar_wait(res_full, 0, abort_flag);
+      // Per query tile it (stage st): S^T = K Q^T and dP^T = V dO^T (M = 128
+      // keys, N = 128 queries, K = D), then, once the compute warps have left
+      // P^T and dS^T in TMEM, dV += P^T dO and dK += dS^T Q (M = 128 keys, N =
+      // D, K = 128 queries; A from TMEM, B the query-side tile, MN-major).
+      // The next tile's S^T goes right after dV (which read the P^T it
+      // overwrites) and its dP^T right after dK, so the compute warps start
+      // the next tile's exponentials while dK and dP^T still run.  One thread
+      // issues everything, in order.
+      auto issue_s = [&](int st) {
+        issue_qk<D>(tmem + kColS, dk_k, hi | sdesc_lo(sQ(st), 16));
+        mma_commit(s_full);
+      };
+      auto issue_dp = [&](int st) {
+        issue_qk<D>(tmem + kColDP, dv_k, hi | sdesc_lo(sDO(st), 16));
+        mma_commit(dp_full);
+      };
+      if (ok && mbar_wait(st_full(0), 0, abort_flag)) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
+      } else {
+        ok = false;
+      }
       for (int it = 0; ok && it < n_it; ++it) {
         const int st = it % kBwdStages;
-        if (!mbar_wait(st_full(st), (it / kBwdStages) & 1, abort_flag)) break;
-        tc_fence_after();
-        // S^T = K Q^T, dP^T = V dO^T (M = 128 keys, N = 128 queries, K = D).
-        // They overwrite P^T, dS^T of the previous tile only after the MMAs
-        // reading them: one thread issues all MMAs, in order.
-        issue_qk<D>(tmem + kColS, dk_k, hi | sdesc_lo(sQ(st), 16));
-        issue_qk<D>(tmem + kColDP, dv_k, hi | sdesc_lo(sDO(st), 16));
-        mma_commit(s_full);
+        const bool next = it + 1 < n_it;
+        const int st1 = (it + 1) % kBwdStages;
         if (!mbar_wait(p_full, it & 1, abort_flag)) break;
+        if (next && !mbar_wait(st_full(st1), ((it + 1) / kBwdStages) & 1, abort_flag)) break;
         tc_fence_after();
-        // dV += P^T dO, dK += dS^T Q (M = 128 keys, N = D, K = 128 queries;
-        // A from TMEM, B = the query-side tile, MN-major).
         const uint64_t ddo_mn = hi | sdesc_lo(sDO(st), Cfg::kBlockBytes);
         const uint64_t dq_mn = hi | sdesc_lo(sQ(st), Cfg::kBlockBytes);
         // P^T, dS^T of queries 0..63 are at columns 0..31 of S^T / dP^T and of
@@ -277,9 +308,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         // of its base, so the second half's base is 32 columns further.
         issue_pv<D, 0>(tmem + kColDV, tmem + kColS, ddo_mn, it > 0);
         issue_pv<D, 1>(tmem + kColDV, tmem + kColS + 32, ddo_mn, true);
+        if (next) issue_s(st1);
         issue_pv<D, 0>(tmem + kColDK, tmem + kColDP, dq_mn, it > 0);
         issue_pv<D, 1>(tmem + kColDK, tmem + kColDP + 32, dq_mn, true);
         mma_commit(st_empty(st));
+        if (next) issue_dp(st1);
       }
       mma_commit(done);
       mbar_wait_drain(done, 0);
@@ -315,15 +348,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       tc_fence_after();
       const float* l2v = l2_at(st);
       const float* ddv = dd_at(st);
-#pragma unroll 1
+      // pass 1, once S^T is in: P (kept) and P^T over S^T's columns 16 h ..
+      // 16 h + 15 of this half (read in step 0 already)
+      float pr[2][32];
+#pragma unroll
       for (int h = 0; h < 2; ++h) {
-        uint32_t sv[32], dp[32], pk[16], dk16[16];
+        uint32_t sv[32], pk[16];
         tmem_ld32(tS + 32 * h, sv);
+        tmem_wait_ld();
+        p_chunk(sv, l2v, 64 * wg + 32 * h, cmin, c, pr[h], pk);
+        tmem_st16(tS + 16 * h, pk);
+      }
+      // pass 2, once dP^T is in: dS^T over dP^T's columns the same way
+      ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t dp[32], dk16[16];
         tmem_ld32(tDP + 32 * h, dp);
         tmem_wait_ld();
-        dkdv_chunk(sv, dp, l2v, ddv, 64 * wg + 32 * h, cmin, c, pk, dk16);
-        // columns 16 h .. 16 h + 15 of this half: read in step 0 already
-        tmem_st16(tS + 16 * h, pk);
+        ds_chunk(pr[h], dp, ddv, 64 * wg + 32 * h, dk16);
         tmem_st16(tDP + 16 * h, dk16);
       }
       tmem_wait_st();
@@ -396,6 +441,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
   const uint32_t p_full = s_full + 8u;
   const uint32_t done = p_full + 8u;
   const uint32_t ds_free = done + 8u;  // dQ += dS K of the previous key tile is done
+  const uint32_t dp_full = ds_free + 8u;  // dP of the current key tile done
   uint8_t* bar_ptr = smem + 2 * Cfg::kTileBytes + kBwdStages * Cfg::kStageBytes;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * Cfg::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -425,6 +471,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
     mbar_init(p_full, kBwdComputeWarps);
     mbar_init(done, 1);
     mbar_init(ds_free, 1);
+    mbar_init(dp_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -467,10 +514,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       const uint64_t hi = static_cast<uint64_t>(sdesc_hi(1024)) << 32;
       const uint64_t dq_k = hi | sdesc_lo(sQ, 16);
       const uint64_t ddo_k = hi | sdesc_lo(sDO, 16);
-      auto issue_s_dp = [&](int st) {  // S = Q K^T, dP = dO V^T (M = 128 queries, N = 128 keys, K = D)
+      // S = Q K^T, then dP = dO V^T (M = 128 queries, N = 128 keys, K = D),
+      // each with its own commit: the compute warps take the exponentials of
+      // S while dP still runs
+      auto issue_s_dp = [&](int st) {
         issue_qk<D>(tmem + kColS, dq_k, hi | sdesc_lo(sK(st), 16));
-        issue_qk<D>(tmem + kColDP, ddo_k, hi | sdesc_lo(sV(st), 16));
         mma_commit(s_full);
+        issue_qk<D>(tmem + kColDP, ddo_k, hi | sdesc_lo(sV(st), 16));
+        mma_commit(dp_full);
       };
       bool ok = mbar_wait(res_full, 0, abort_flag) && mbar_wait(st_full(0), 0, abort_flag);
       if (ok) {
@@ -515,25 +566,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
+      // pass 1, once S is in: P (fp32)
+      float pr[2][32];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int ch = 2 * wg + h;
+        uint32_t sv[32];
+        tmem_ld32(tmem + lane_bits + kColS + ch * 32, sv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int col = ch * 32 + e;
+          pr[h][e] = (col <= jlim) ? ex2_approx(fmaf(__uint_as_float(sv[e]), c, -l2)) : 0.f;
+        }
+      }
+      // pass 2, once dP is in: dS = P (dP - D)
+      ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
       uint32_t pk[2][16];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int ch = 2 * wg + h;
-        uint32_t sv[32], dp[32];
-        tmem_ld32(tmem + lane_bits + kColS + ch * 32, sv);
+        uint32_t dp[32];
         tmem_ld32(tmem + lane_bits + kColDP + ch * 32, dp);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = ch * 32 + e + u;
-            const float pr = (col <= jlim) ? ex2_approx(fmaf(__uint_as_float(sv[e + u]), c, -l2)) : 0.f;
-            ds[u] = pr * (__uint_as_float(dp[e + u]) - dd);
-          }
-          pk[h][e / 2] = pack_bf16x2(ds[0], ds[1]);
-        }
+        for (int e = 0; e < 32; e += 2)
+          pk[h][e / 2] = pack_bf16x2(pr[h][e] * (__uint_as_float(dp[e]) - dd),
+                                     pr[h][e + 1] * (__uint_as_float(dp[e + 1]) - dd));
       }
       // the dS columns are free once dQ += dS K of the previous key tile is done
       if (it > 0) {
