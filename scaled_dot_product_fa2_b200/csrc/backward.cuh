@@ -97,9 +97,10 @@ struct BwdCfg {
   static constexpr int kVecBytes = 128 * 4;         // 128 fp32 (L2 or D of one query tile)
   // smem: two resident tiles, then per stage two streamed tiles and two vectors
   static constexpr int kStageBytes = 2 * kTileBytes + 2 * kVecBytes;
-  // res_full, st_full[2], st_empty[2], s_full, p_full, done, then dK/dV: dp_full;
-  // dQ: ds_free (the previous dS has been read), dp_full
-  static constexpr int kNumBars = 1 + 2 * kBwdStages + 5;
+  // res_full, st_full[2], st_empty[2], s_full, p_full, done, then dK/dV: dp_full
+  // (and ds_full); dQ: ds_free (the previous dS has been read), dp_full, s_free,
+  // dp_free (S / dP read out of TMEM)
+  static constexpr int kNumBars = 1 + 2 * kBwdStages + 7;
   static constexpr int kSmemBytes = 2 * kTileBytes + kBwdStages * kStageBytes + kNumBars * 8 + 16 + 1024;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
   static constexpr uint32_t kTmemCols = 512;
@@ -196,6 +197,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
   const uint32_t p_full = s_full + 8u;
   const uint32_t done = p_full + 8u;
   const uint32_t dp_full = done + 8u;  // dP^T of the current query tile done
+  const uint32_t ds_full = dp_full + 8u;  // dS^T of the current query tile written (p_full: P^T)
   uint8_t* bar_ptr = smem + 2 * Cfg::kTileBytes + kBwdStages * Cfg::kStageBytes;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * Cfg::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -222,6 +224,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     mbar_init(p_full, kBwdComputeWarps);  // one arrive per compute warp
     mbar_init(done, 1);
     mbar_init(dp_full, 1);
+    mbar_init(ds_full, kBwdComputeWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -272,13 +275,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       const uint64_t dv_k = hi | sdesc_lo(sV, 16);  // V, K-major (A of dP^T)
       bool ok = mbar_wait(res_full, 0, abort_flag);
       // Per query tile it (stage st): S^T = K Q^T and dP^T = V dO^T (M = 128
-      // keys, N = 128 queries, K = D), then, once the compute warps have left
-      // P^T and dS^T in TMEM, dV += P^T dO and dK += dS^T Q (M = 128 keys, N =
-      // D, K = 128 queries; A from TMEM, B the query-side tile, MN-major).
-      // The next tile's S^T goes right after dV (which read the P^T it
-      // overwrites) and its dP^T right after dK, so the compute warps start
-      // the next tile's exponentials while dK and dP^T still run.  One thread
-      // issues everything, in order.
+      // keys, N = 128 queries, K = D); dV += P^T dO once the compute warps
+      // have left P^T in TMEM, and dK += dS^T Q once they have left dS^T
+      // (M = 128 keys, N = D, K = 128 queries; A from TMEM, B the query-side
+      // tile, MN-major).  The next tile's S^T goes right after dV (which read
+      // the P^T it overwrites) and its dP^T right after dK, so the compute
+      // warps' dS^T overlaps dV and the next S^T, and their next exponentials
+      // overlap dK and the next dP^T.  One thread issues everything, in order.
       auto issue_s = [&](int st) {
         issue_qk<D>(tmem + kColS, dk_k, hi | sdesc_lo(sQ(st), 16));
         mma_commit(s_full);
@@ -309,6 +312,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         issue_pv<D, 0>(tmem + kColDV, tmem + kColS, ddo_mn, it > 0);
         issue_pv<D, 1>(tmem + kColDV, tmem + kColS + 32, ddo_mn, true);
         if (next) issue_s(st1);
+        if (!mbar_wait(ds_full, it & 1, abort_flag)) break;
+        tc_fence_after();
         issue_pv<D, 0>(tmem + kColDK, tmem + kColDP, dq_mn, it > 0);
         issue_pv<D, 1>(tmem + kColDK, tmem + kColDP + 32, dq_mn, true);
         mma_commit(st_empty(st));
@@ -359,6 +364,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         p_chunk(sv, l2v, 64 * wg + 32 * h, cmin, c, pr[h], pk);
         tmem_st16(tS + 16 * h, pk);
       }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);  // P^T written: dV may run
       // pass 2, once dP^T is in: dS^T over dP^T's columns the same way
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag));
       if (!ok) break;
@@ -374,7 +383,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(ds_full);  // dS^T written: dK may run
     }
     // ---- epilogue: dK = scale * acc, dV = acc -> bf16 rows.  The TMEM loads
     // are collective: the whole warp runs them (warp-uniform `have`); only
@@ -440,8 +449,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
   const uint32_t s_full = bar0 + 8u * (1 + 2 * kBwdStages);
   const uint32_t p_full = s_full + 8u;
   const uint32_t done = p_full + 8u;
-  const uint32_t ds_free = done + 8u;  // dQ += dS K of the previous key tile is done
+  const uint32_t ds_free = done + 8u;     // dQ += dS K of the previous key tile is done
   const uint32_t dp_full = ds_free + 8u;  // dP of the current key tile done
+  const uint32_t s_free = dp_full + 8u;   // every compute warp has read S of the current key tile
+  const uint32_t dp_free = s_free + 8u;   // ... and dP
   uint8_t* bar_ptr = smem + 2 * Cfg::kTileBytes + kBwdStages * Cfg::kStageBytes;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * Cfg::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -472,6 +483,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
     mbar_init(done, 1);
     mbar_init(ds_free, 1);
     mbar_init(dp_full, 1);
+    mbar_init(s_free, kBwdComputeWarps);
+    mbar_init(dp_free, kBwdComputeWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -514,28 +527,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       const uint64_t hi = static_cast<uint64_t>(sdesc_hi(1024)) << 32;
       const uint64_t dq_k = hi | sdesc_lo(sQ, 16);
       const uint64_t ddo_k = hi | sdesc_lo(sDO, 16);
-      // S = Q K^T, then dP = dO V^T (M = 128 queries, N = 128 keys, K = D),
-      // each with its own commit: the compute warps take the exponentials of
-      // S while dP still runs
-      auto issue_s_dp = [&](int st) {
+      // Key tile it+1's S = Q K^T (M = 128 queries, N = 128 keys, K = D) is
+      // issued as soon as the compute warps have read tile it's S out of TMEM
+      // (they keep P in registers), its dP = dO V^T once they have read tile
+      // it's dP, and dQ += dS K for tile it once its dS is written: the
+      // tensor core computes the next tile's S while the compute warps still
+      // take this tile's exponentials.
+      auto issue_s = [&](int st) {
         issue_qk<D>(tmem + kColS, dq_k, hi | sdesc_lo(sK(st), 16));
         mma_commit(s_full);
+      };
+      auto issue_dp = [&](int st) {
         issue_qk<D>(tmem + kColDP, ddo_k, hi | sdesc_lo(sV(st), 16));
         mma_commit(dp_full);
       };
       bool ok = mbar_wait(res_full, 0, abort_flag) && mbar_wait(st_full(0), 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        issue_s_dp(0);
+        issue_s(0);
+        issue_dp(0);
       }
       for (int it = 0; ok && it < n_it; ++it) {
         const int st = it % kBwdStages;
-        // dS(it) written (S, dP of tile it no longer needed), next tile landed
-        if (!mbar_wait(p_full, it & 1, abort_flag)) break;
         const bool next = it + 1 < n_it;
-        if (next && !mbar_wait(st_full((it + 1) % kBwdStages), ((it + 1) / kBwdStages) & 1, abort_flag)) break;
+        const int st1 = (it + 1) % kBwdStages;
+        if (next) {
+          if (!mbar_wait(s_free, it & 1, abort_flag) ||
+              !mbar_wait(st_full(st1), ((it + 1) / kBwdStages) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_s(st1);
+          if (!mbar_wait(dp_free, it & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_dp(st1);
+        }
+        // dS(it) written
+        if (!mbar_wait(p_full, it & 1, abort_flag)) break;
         tc_fence_after();
-        if (next) issue_s_dp((it + 1) % kBwdStages);
         // dQ += dS K (M = 128 queries, N = D, K = 128 keys; dS from TMEM, K MN-major)
         const uint64_t dk_mn = hi | sdesc_lo(sK(st), Cfg::kBlockBytes);
         issue_pv<D, 0>(tmem + kColDQ, tmem + kColDS, dk_mn, it > 0);
@@ -574,6 +607,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
         uint32_t sv[32];
         tmem_ld32(tmem + lane_bits + kColS + ch * 32, sv);
         tmem_wait_ld();
+        if (h == 1) {  // this warp's part of S is read: the next key tile's S may overwrite it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free);
+        }
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int col = ch * 32 + e;
@@ -591,6 +629,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
         uint32_t dp[32];
         tmem_ld32(tmem + lane_bits + kColDP + ch * 32, dp);
         tmem_wait_ld();
+        if (h == 1) {  // this warp's part of dP is read
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(dp_free);
+        }
 #pragma unroll
         for (int e = 0; e < 32; e += 2)
           pk[h][e / 2] = pack_bf16x2(pr[h][e] * (__uint_as_float(dp[e]) - dd),
