@@ -128,3 +128,35 @@ def test_decode_bias_with_per_batch_lengths(sdpa):
                                       v[b:b + 1, :, :L].double().numpy(), 1 / math.sqrt(d), BR,
                                       bias=bias[b:b + 1, :, :, :L].double().numpy())
         parity.compare(o[b:b + 1], lse[b:b + 1], o_ref, lse_ref, f"batch {b}")
+
+
+@pytest.mark.parametrize("causal", [TL, BR])
+def test_forward_bias_with_per_batch_lengths(sdpa, causal):
+    """Bias and per-batch lengths together (attn_fwd_ex with both extras):
+    the run-time unit hand-out and the bias loader walk the same units; each
+    batch's valid rows equal the oracle on its own rows, keys and bias block."""
+    import ctypes
+    from scaled_dot_product_fa2_b200 import _lib
+    B, Hq, Hkv, S, d = 3, 4, 2, 600, 128
+    lq, lk = [600, 130, 257], [600, 416, 257]
+    q, k, v = parity.seeded(B, Hq, Hkv, S, S, d, seed=940 + causal)
+    bias = make_bias((1, Hq), S, S, seed=941 + causal)
+    qd, kd, vd = parity.to_dev(q, k, v)
+    o, lse = parity.nan_outputs(qd, B, Hq, S)
+    bd = bias.cuda()
+    sq = torch.tensor(lq, dtype=torch.int32, device="cuda")
+    sk = torch.tensor(lk, dtype=torch.int32, device="cuda")
+    ex = _lib.Extras()
+    ex.seqlens_q, ex.seqlens_k, ex.bias = sq.data_ptr(), sk.data_ptr(), bd.data_ptr()
+    ex.bias_b, ex.bias_h, ex.layout = 1, Hq, 0
+    st = _lib.get().attn_fwd_ex(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv,
+                                S, S, d, 0.0, causal, ctypes.byref(ex), torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    sdpa.check_device_error()
+    o = o.float().cpu().numpy()
+    lse = lse.cpu().numpy()
+    for b in range(B):
+        assert np.isnan(o[b, :, lq[b]:]).all(), f"batch {b}: padding rows written"
+        o_ref, lse_ref = oracle(q[b:b + 1, :, :lq[b]], k[b:b + 1, :, :lk[b]], v[b:b + 1, :, :lk[b]],
+                                bias[:, :, :lq[b], :lk[b]].contiguous(), causal, d)
+        parity.compare(o[b:b + 1, :, :lq[b]], lse[b:b + 1, :, :lq[b]], o_ref, lse_ref, f"bias varlen batch {b}")
