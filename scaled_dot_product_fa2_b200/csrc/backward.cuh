@@ -27,7 +27,9 @@
 //                     dK, each with its own commit, so its P^T (the
 //                     exponentials) is under way while dK and dP^T run.
 //   bwd_dq_kernel     one CTA per 128-row query tile: Q and dO stay in shared
-//                     memory while the key tiles stream; S = Q K^T and
+//                     memory while the key tiles stream through a ring of
+//                     single K and V slots (V_j freed after dP_j, K_j after
+//                     dS_j K_j, so the next tiles land early); S = Q K^T and
 //                     dP = dO V^T, dS by the compute warps into TMEM columns
 //                     of its own, dQ += dS K.  With dS apart from S, the next
 //                     tile's S and dP are issued before this tile's dS K, and
@@ -103,6 +105,16 @@ struct BwdCfg {
   static constexpr int kNumBars = 1 + 2 * kBwdStages + 7;
   static constexpr int kSmemBytes = 2 * kTileBytes + kBwdStages * kStageBytes + kNumBars * 8 + 16 + 1024;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
+  // dQ kernel: Q, dO resident, then a ring of kDqSlots single tiles (K_0, V_0,
+  // K_1, V_1, ...): V_j's slot is free once dP_j is done and K_j's once
+  // dQ += dS_j K_j is, so the next tiles start landing a whole tile earlier
+  // than with K and V in one stage; then res_full, kv_full[kDqSlots],
+  // kv_empty[kDqSlots], s_full, p_full, done, ds_free, dp_full, s_free, dp_free
+  static constexpr int kDqSlots = D == 128 ? 5 : 8;
+  static constexpr int kDqNumBars = 1 + 2 * kDqSlots + 7;
+  static constexpr int kDqSmemBytes = (2 + kDqSlots) * kTileBytes + kDqNumBars * 8 + 16 + 1024;
+  static_assert(kDqSmemBytes <= 227 * 1024, "shared memory per block");
+  static constexpr int kDqSmemLaunch = kDqSmemBytes > 116 * 1024 ? kDqSmemBytes : 116 * 1024;
   static constexpr uint32_t kTmemCols = 512;
   // Each CTA takes all 512 TMEM columns, and tcgen05.alloc waits without a
   // bound for columns another CTA holds: launch with more than half of the
@@ -437,24 +449,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
   using Cfg = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // Q | dO | stage 0: K, V (vector space unused) | stage 1 | barriers
+  // Q | dO | ring of kDqSlots tiles: position 2j holds K_j, 2j + 1 holds V_j | barriers
+  constexpr int NSL = Cfg::kDqSlots;
   const uint32_t sQ = smem_u32(smem);
   const uint32_t sDO = sQ + Cfg::kTileBytes;
-  auto sK = [&](int st) { return sQ + 2 * Cfg::kTileBytes + st * Cfg::kStageBytes; };
-  auto sV = [&](int st) { return sK(st) + Cfg::kTileBytes; };
-  const uint32_t bar0 = sQ + 2 * Cfg::kTileBytes + kBwdStages * Cfg::kStageBytes;
+  auto slot_addr = [&](int pos) { return sQ + (2 + pos % NSL) * Cfg::kTileBytes; };
+  const uint32_t bar0 = sQ + (2 + NSL) * Cfg::kTileBytes;
   const uint32_t res_full = bar0;
-  auto st_full = [&](int st) { return bar0 + 8u * (1 + st); };
-  auto st_empty = [&](int st) { return bar0 + 8u * (1 + kBwdStages + st); };
-  const uint32_t s_full = bar0 + 8u * (1 + 2 * kBwdStages);
+  auto kv_full = [&](int pos) { return bar0 + 8u * (1 + pos % NSL); };
+  auto kv_empty = [&](int pos) { return bar0 + 8u * (1 + NSL + pos % NSL); };
+  auto kv_par = [&](int pos) { return static_cast<uint32_t>((pos / NSL) & 1); };
+  const uint32_t s_full = bar0 + 8u * (1 + 2 * NSL);
   const uint32_t p_full = s_full + 8u;
   const uint32_t done = p_full + 8u;
   const uint32_t ds_free = done + 8u;     // dQ += dS K of the previous key tile is done
   const uint32_t dp_full = ds_free + 8u;  // dP of the current key tile done
   const uint32_t s_free = dp_full + 8u;   // every compute warp has read S of the current key tile
   const uint32_t dp_free = s_free + 8u;   // ... and dP
-  uint8_t* bar_ptr = smem + 2 * Cfg::kTileBytes + kBwdStages * Cfg::kStageBytes;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * Cfg::kNumBars);
+  uint8_t* bar_ptr = smem + (2 + NSL) * Cfg::kTileBytes;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * Cfg::kDqNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -474,9 +487,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
 
   if (threadIdx.x == 0) {
     mbar_init(res_full, 1);
-    for (int st = 0; st < kBwdStages; ++st) {
-      mbar_init(st_full(st), 1);
-      mbar_init(st_empty(st), 1);
+    for (int sl = 0; sl < NSL; ++sl) {
+      mbar_init(kv_full(sl), 1);
+      mbar_init(kv_empty(sl), 1);
     }
     mbar_init(s_full, 1);
     mbar_init(p_full, kBwdComputeWarps);
@@ -508,18 +521,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
         tma_load_4d(sQ + blk * Cfg::kBlockBytes, &p.tm_q, blk * 64, i0, hq, b, res_full);
         tma_load_4d(sDO + blk * Cfg::kBlockBytes, &p.tm_do, blk * 64, i0, hq, b, res_full);
       }
-      int it = 0;
-      for (; it < n_it; ++it) {
-        const int st = it % kBwdStages;
-        if (!mbar_wait(st_empty(st), ((it / kBwdStages) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(st_full(st), 2 * Cfg::kTileBytes);
-        for (int blk = 0; blk < Cfg::kBlocks; ++blk) {
-          tma_load_4d(sK(st) + blk * Cfg::kBlockBytes, &p.tm_k, blk * 64, it * 128, hkv, b, st_full(st));
-          tma_load_4d(sV(st) + blk * Cfg::kBlockBytes, &p.tm_v, blk * 64, it * 128, hkv, b, st_full(st));
-        }
+      int pos = 0;  // ring positions issued: K_j at 2j, V_j at 2j + 1
+      for (; pos < 2 * n_it; ++pos) {
+        if (!mbar_wait(kv_empty(pos), kv_par(pos) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(kv_full(pos), Cfg::kTileBytes);
+        const CUtensorMap* tm = (pos & 1) ? &p.tm_v : &p.tm_k;
+        for (int blk = 0; blk < Cfg::kBlocks; ++blk)
+          tma_load_4d(slot_addr(pos) + blk * Cfg::kBlockBytes, tm, blk * 64, (pos >> 1) * 128, hkv, b, kv_full(pos));
       }
       mbar_wait_drain(res_full, 0);
-      for (int i = max(0, it - kBwdStages); i < it; ++i) mbar_wait_drain(st_full(i % kBwdStages), (i / kBwdStages) & 1);
+      for (int i = max(0, pos - NSL); i < pos; ++i) mbar_wait_drain(kv_full(i), kv_par(i));
     }
     __syncwarp();
   } else if (warp == kBwdMmaWarp) {
@@ -533,48 +544,51 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       // it's dP, and dQ += dS K for tile it once its dS is written: the
       // tensor core computes the next tile's S while the compute warps still
       // take this tile's exponentials.
-      auto issue_s = [&](int st) {
-        issue_qk<D>(tmem + kColS, dq_k, hi | sdesc_lo(sK(st), 16));
+      // S(j) reads K_j (ring position 2j), dP(j) V_j (2j + 1), dQ(j) K_j
+      // again; V_j's slot is released after dP(j), K_j's after dQ(j).
+      auto issue_s = [&](int j) {
+        issue_qk<D>(tmem + kColS, dq_k, hi | sdesc_lo(slot_addr(2 * j), 16));
         mma_commit(s_full);
       };
-      auto issue_dp = [&](int st) {
-        issue_qk<D>(tmem + kColDP, ddo_k, hi | sdesc_lo(sV(st), 16));
+      auto issue_dp = [&](int j) {
+        issue_qk<D>(tmem + kColDP, ddo_k, hi | sdesc_lo(slot_addr(2 * j + 1), 16));
         mma_commit(dp_full);
+        mma_commit(kv_empty(2 * j + 1));
       };
-      bool ok = mbar_wait(res_full, 0, abort_flag) && mbar_wait(st_full(0), 0, abort_flag);
+      bool ok = mbar_wait(res_full, 0, abort_flag) && mbar_wait(kv_full(0), kv_par(0), abort_flag) &&
+                mbar_wait(kv_full(1), kv_par(1), abort_flag);
       if (ok) {
         tc_fence_after();
         issue_s(0);
         issue_dp(0);
       }
       for (int it = 0; ok && it < n_it; ++it) {
-        const int st = it % kBwdStages;
         const bool next = it + 1 < n_it;
-        const int st1 = (it + 1) % kBwdStages;
         if (next) {
           if (!mbar_wait(s_free, it & 1, abort_flag) ||
-              !mbar_wait(st_full(st1), ((it + 1) / kBwdStages) & 1, abort_flag)) {
+              !mbar_wait(kv_full(2 * it + 2), kv_par(2 * it + 2), abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_s(st1);
-          if (!mbar_wait(dp_free, it & 1, abort_flag)) {
+          issue_s(it + 1);
+          if (!mbar_wait(dp_free, it & 1, abort_flag) ||
+              !mbar_wait(kv_full(2 * it + 3), kv_par(2 * it + 3), abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_dp(st1);
+          issue_dp(it + 1);
         }
         // dS(it) written
         if (!mbar_wait(p_full, it & 1, abort_flag)) break;
         tc_fence_after();
         // dQ += dS K (M = 128 queries, N = D, K = 128 keys; dS from TMEM, K MN-major)
-        const uint64_t dk_mn = hi | sdesc_lo(sK(st), Cfg::kBlockBytes);
+        const uint64_t dk_mn = hi | sdesc_lo(slot_addr(2 * it), Cfg::kBlockBytes);
         issue_pv<D, 0>(tmem + kColDQ, tmem + kColDS, dk_mn, it > 0);
         issue_pv<D, 1>(tmem + kColDQ, tmem + kColDS, dk_mn, true);
         mma_commit(ds_free);
-        mma_commit(st_empty(st));
+        mma_commit(kv_empty(2 * it));
       }
       mma_commit(done);
       mbar_wait_drain(done, 0);

@@ -382,7 +382,7 @@ attn_status_t launch_bwd(const BwdParams& prm, int dev, cudaStream_t st) {
   {
     std::lock_guard<std::mutex> lock(mu);
     if (!set_smem(bwd_dkdv_kernel<D>, Cfg::kSmemLaunch, dev, smem_done_kv) ||
-        !set_smem(bwd_dq_kernel<D>, Cfg::kSmemLaunch, dev, smem_done_q))
+        !set_smem(bwd_dq_kernel<D>, Cfg::kDqSmemLaunch, dev, smem_done_q))
       return ATTN_ERR_CUDA;
   }
   const int64_t prep_rows = static_cast<int64_t>(prm.B) * prm.Hq * prm.Sq_pad;
@@ -395,7 +395,7 @@ attn_status_t launch_bwd(const BwdParams& prm, int dev, cudaStream_t st) {
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   if (g_q > 0) {
-    bwd_dq_kernel<D><<<static_cast<unsigned>(g_q), kBwdThreads, Cfg::kSmemLaunch, st>>>(prm);
+    bwd_dq_kernel<D><<<static_cast<unsigned>(g_q), kBwdThreads, Cfg::kDqSmemLaunch, st>>>(prm);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
