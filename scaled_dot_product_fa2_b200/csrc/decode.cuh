@@ -102,6 +102,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
   auto empty = [&](int s) { return bar0 + 8u * (NSTAGE + s); }; // [NSTAGE] stage released
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kRingBytes + 16 * NSTAGE);
 
+  // Launched as a programmatic dependent of the previous kernel in the
+  // stream (the previous call's combine, in a decode loop): this grid's CTAs
+  // may be resident before that kernel ends, and wait here, before any global
+  // memory access, for its completion and the visibility of its writes.
+  grid_dependency_wait();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int rg = static_cast<int>(blockIdx.x) % p.row_groups;
@@ -408,6 +413,8 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
   constexpr int kPer = D / 32;  // floats per lane: 4 (one 16-byte load) or 2
   constexpr int kUnroll = 8;
   constexpr float kLog2e = 1.4426950408889634f;
+  // the next kernel in the stream (a programmatic dependent) may be scheduled now
+  grid_dependency_trigger();
   grid_dependency_wait();
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);

@@ -343,11 +343,20 @@ attn_status_t launch_decode(const DecodeParams& prm, int grid, float* part_o, fl
     std::lock_guard<std::mutex> lock(mu);
     if (!set_smem(decode_split_kernel<D, kDecStages>, Cfg::kSmemBytes, dev, smem_done)) return ATTN_ERR_CUDA;
   }
+  // The split kernel is itself a programmatic dependent of whatever precedes
+  // it in the stream: its CTAs can be resident while that kernel finishes and
+  // wait (griddepcontrol.wait) before touching global memory, which hides the
+  // launch between back-to-back decode calls.
+  cudaLaunchAttribute sattr[1];
+  sattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  sattr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kDecThreads);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = st;
+  cfg.attrs = sattr;
+  cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, decode_split_kernel<D, kDecStages>, prm) != cudaSuccess) return ATTN_ERR_CUDA;
   // The combine is a programmatic dependent launch: it may be scheduled while
   // the split kernel's last CTAs run and waits (griddepcontrol.wait) for the
