@@ -11,9 +11,13 @@
 // Sq rows, up to 16 per CTA).
 //
 // B200 mapping (this file's own design):
-//   * grid = (row group, split, batch*kv_head); 4 consumer warps + 1 TMA
-//     producer warp; K/V tiles of 64 keys stream through an NSTAGE-deep ring
-//     of 128-byte-swizzled shared-memory tiles.
+//   * grid = (kv head, slot, row group); 4 consumer warps + 1 TMA producer
+//     warp; K/V tiles of 64 keys stream through an NSTAGE-deep ring of
+//     128-byte-swizzled shared-memory tiles.
+//   * A KV head has B * nsplit slots (CTAs).  With one cache length every
+//     batch takes nsplit of them; with per-batch lengths the slots are dealt
+//     in proportion to each batch's tiles (assign_slot), so a mix of long and
+//     short caches keeps every CTA's share of the keys about equal.
 //   * The work per byte is tiny (<= 16 query rows), so the contraction runs on
 //     warp-level mma.sync m16n8k16 (bf16, fp32 accumulate): the kernel is
 //     bound by HBM bandwidth, not by the tensor pipe.  Each warp owns 16 keys
@@ -35,8 +39,8 @@ struct DecodeParams {
   const uint16_t* bias;   // bf16 additive bias [bias_b][bias_h][Sq][Sk], or nullptr
   int64_t bias_sb, bias_sh;  // its batch and head strides in elements (0 where it broadcasts)
   float inv_scale;        // 1 / scale: the bias enters the raw scores as bias / scale
-  float* part_o;          // [B*Hq*Sq][nsplit][d]  locally normalised partial outputs
-  float2* part_ml;        // [B*Hq*Sq][nsplit]     (local max of scale*q.k, local sum)
+  float* part_o;          // [Hkv][B*nsplit slots][G*Sq rows][d]  locally normalised partial outputs
+  float2* part_ml;        // [Hkv][B*nsplit slots][G*Sq rows]     (local max of scale*q.k, local sum)
   int B, Hq, Hkv, Sq, Sk, group;
   int causal;             // 0 none, 1 top-left, 2 bottom-right
   int causal_offset;      // key j visible to row i iff j <= i + causal_offset (if causal; fixed-length caches)
@@ -91,6 +95,116 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c, int block_bytes) {
   return (c >> 6) * block_bytes + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1);
 }
 
+// Slot deal for per-batch key lengths.  A KV head has `slots` CTAs
+// (B * nsplit).  Batch b has T_b = ceil(len_b / 64) tiles; the per-CTA quota
+// q is the smallest number of tiles for which sum_b max(1, ceil(T_b / q))
+// slots suffice, and batch b takes n_b = max(1, ceil(T_b / q)) consecutive
+// slots, its k-th slot streaming tiles [k q, min(T_b, (k + 1) q)).  So the
+// longest CTA does as little as whole tiles allow, whatever the length mix;
+// an empty batch still gets one slot (it writes o = 0, lse = -inf).  The
+// split kernel (slot -> batch) and the combine (batch -> slots) both derive
+// the deal from the lengths; every lane of the calling warp gets the same
+// answer.
+__device__ __forceinline__ int len_tiles(const int* __restrict__ seqlens, int bb, int B, int Sk) {
+  return bb < B ? (min(max(__ldg(seqlens + bb), 0), Sk) + kDecKeys - 1) / kDecKeys : 0;
+}
+
+__device__ __forceinline__ int64_t warp_sum_i64(int64_t v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+// Inclusive prefix sum over the warp.
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += u;
+  }
+  return v;
+}
+
+// The quota q.  t0 = len_tiles(lane): the first 32 batches stay in a register.
+__device__ __forceinline__ int slot_quota(const int* __restrict__ seqlens, int B, int Sk, int slots, int lane,
+                                          int t0) {
+  auto tiles_at = [&](int b0) { return b0 == 0 ? t0 : len_tiles(seqlens, b0 + lane, B, Sk); };
+  int64_t tot = 0;
+  int mx = 0;
+  for (int b0 = 0; b0 < B; b0 += 32) {
+    const int t = tiles_at(b0);
+    tot += t;
+    mx = max(mx, t);
+  }
+  tot = warp_sum_i64(tot);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  auto fits = [&](int q) {
+    int64_t n = 0;
+    for (int b0 = 0; b0 < B; b0 += 32)
+      if (b0 + lane < B) n += max(1, (tiles_at(b0) + q - 1) / q);
+    return warp_sum_i64(n) <= slots;
+  };
+  // No q below ceil(tot / slots) fits; q = max T_b always does (B <= slots),
+  // and so does ceil(tot / (slots - B)), since max(1, ceil(T_b / q)) <= T_b / q + 1.
+  // Equal lengths fit at the lower bound: it is tried first.
+  const int64_t lo0 = (tot + slots - 1) / slots;
+  int lo = lo0 > 1 ? static_cast<int>(lo0) : 1;
+  int hi = max(1, mx);
+  if (slots > B) hi = min(hi, max(lo, static_cast<int>((tot + (slots - B) - 1) / (slots - B))));
+  if (lo < hi && fits(lo)) hi = lo;
+  else if (lo < hi) ++lo;
+  while (lo < hi) {
+    const int mid = lo + ((hi - lo) >> 1);
+    if (fits(mid)) hi = mid;
+    else lo = mid + 1;
+  }
+  return lo;
+}
+
+struct SlotAssign {
+  int b, k, quota;  // b = -1: a slot that no batch needs
+};
+
+__device__ __forceinline__ SlotAssign assign_slot(const int* __restrict__ seqlens, int B, int Sk, int slots, int j,
+                                                  int lane) {
+  const int t0 = len_tiles(seqlens, lane, B, Sk);
+  const int q = slot_quota(seqlens, B, Sk, slots, lane, t0);
+  int start = 0;
+  for (int b0 = 0; b0 < B; b0 += 32) {
+    const int t = b0 == 0 ? t0 : len_tiles(seqlens, b0 + lane, B, Sk);
+    const int n = (b0 + lane < B) ? max(1, (t + q - 1) / q) : 0;
+    const int incl = warp_incl_scan(n, lane);
+    const int excl = incl - n;
+    const unsigned hit = __ballot_sync(0xffffffffu, n > 0 && j >= start + excl && j < start + incl);
+    if (hit != 0u) {
+      const int src = __ffs(hit) - 1;
+      return {b0 + src, j - start - __shfl_sync(0xffffffffu, excl, src), q};
+    }
+    start += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  return {-1, 0, q};
+}
+
+// (first slot, slot count) of batch b.
+__device__ __forceinline__ int2 batch_slots(const int* __restrict__ seqlens, int B, int Sk, int slots, int b,
+                                            int lane) {
+  const int t0 = len_tiles(seqlens, lane, B, Sk);
+  const int q = slot_quota(seqlens, B, Sk, slots, lane, t0);
+  int start = 0;
+  for (int b0 = 0; b0 < B; b0 += 32) {
+    const int t = b0 == 0 ? t0 : len_tiles(seqlens, b0 + lane, B, Sk);
+    const int n = (b0 + lane < B) ? max(1, (t + q - 1) / q) : 0;
+    const int incl = warp_incl_scan(n, lane);
+    if (b < b0 + 32) {
+      const int src = b - b0;
+      return make_int2(start + __shfl_sync(0xffffffffu, incl - n, src), __shfl_sync(0xffffffffu, n, src));
+    }
+    start += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  return make_int2(0, 0);
+}
+
 template <int D, int NSTAGE>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_constant__ DecodeParams p) {
   using Cfg = DecodeCfg<D, NSTAGE>;
@@ -101,44 +215,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
   auto full = [&](int s) { return bar0 + 8u * s; };             // [NSTAGE] stage filled
   auto empty = [&](int s) { return bar0 + 8u * (NSTAGE + s); }; // [NSTAGE] stage released
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kRingBytes + 16 * NSTAGE);
-
-  // Launched as a programmatic dependent of the previous kernel in the
-  // stream (the previous call's combine, in a decode loop): this grid's CTAs
-  // may be resident before that kernel ends, and wait here, before any global
-  // memory access, for its completion and the visibility of its writes.
-  grid_dependency_wait();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int rg = static_cast<int>(blockIdx.x) % p.row_groups;
-  const int split = (static_cast<int>(blockIdx.x) / p.row_groups) % p.nsplit;
-  const int bhkv = static_cast<int>(blockIdx.x) / (p.row_groups * p.nsplit);
-  const int b = bhkv / p.Hkv;
-  const int hkv = bhkv - b * p.Hkv;
-  const int rows_total = p.group * p.Sq;  // query rows sharing this KV head
-  // Valid keys of this batch's cache.  With per-batch lengths (read here, on
-  // the device, so the grid never depends on them) this batch's tiles are
-  // spread evenly over the splits, and the mask is aligned to its own length.
-  int L = p.Sk;
-  int tps = p.tiles_per_split;
-  int coff = p.causal_offset;
-  if (p.seqlens_k != nullptr) {
-    const int raw = __ldg(p.seqlens_k + b);
-    L = min(max(raw, 0), p.Sk);
-    if (raw != L && threadIdx.x == 0 && split == 0 && rg == 0 && hkv == 0) atomicOr(&g_error_word, kErrSeqlen);
-    tps = ((L + kDecKeys - 1) / kDecKeys + p.nsplit - 1) / p.nsplit;
-    coff = (p.causal == 2) ? L - p.Sq : 0;
-  }
-  const int total_tiles = (L + kDecKeys - 1) / kDecKeys;
-  const int tile_begin = split * tps;
-  const int tile_end = min(total_tiles, tile_begin + tps);
-  const int ntiles = max(0, tile_end - tile_begin);
-  // first flattened (b*Hq + hq)*Sq + i row of this KV head
-  const int64_t row_base = (static_cast<int64_t>(b) * p.Hq + static_cast<int64_t>(hkv) * p.group) * p.Sq;
 
-  // Let the combine kernel (a programmatic dependent launch) be scheduled
-  // as soon as every CTA of this grid has started; it waits for this grid's
-  // completion before it reads anything.
-  grid_dependency_trigger();
+  // Shared-memory set-up and the tensor-map prefetch touch no global memory
+  // that an earlier kernel writes, so they run before the dependency wait.
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(full(s), 1);
@@ -147,12 +228,58 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     *abort_flag = 0;
     fence_barrier_init();
   }
+  if (warp == kDecProducerWarp && lane == 0) {
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+  }
+  // Launched as a programmatic dependent of the previous kernel in the
+  // stream (the previous call's combine, in a decode loop): this grid's CTAs
+  // may be resident before that kernel ends, and wait here, before any global
+  // memory access, for its completion and the visibility of its writes.
+  grid_dependency_wait();
+
+  // blockIdx.x = (kv head * slots + slot) * row_groups + row group
+  const int slots = p.B * p.nsplit;  // CTAs per (kv head, row group)
+  const int rg = static_cast<int>(blockIdx.x) % p.row_groups;
+  const int j = (static_cast<int>(blockIdx.x) / p.row_groups) % slots;
+  const int hkv = static_cast<int>(blockIdx.x) / (p.row_groups * slots);
+  const int rows_total = p.group * p.Sq;  // query rows sharing this KV head
+  // Batch of this slot, its index among the batch's slots and the tiles it
+  // streams.  One cache length: nsplit slots per batch.  Per-batch lengths
+  // (read here, on the device, so the grid never depends on them): slots are
+  // dealt to batches in proportion to their tiles, and the mask is aligned to
+  // each batch's own length.
+  int b, k_in_batch, tile_begin, tile_end;
+  int L = p.Sk;
+  int coff = p.causal_offset;
+  if (p.seqlens_k == nullptr) {
+    b = j / p.nsplit;
+    k_in_batch = j - b * p.nsplit;
+    tile_begin = k_in_batch * p.tiles_per_split;
+    tile_end = min((L + kDecKeys - 1) / kDecKeys, tile_begin + p.tiles_per_split);
+  } else {
+    const SlotAssign a = assign_slot(p.seqlens_k, p.B, p.Sk, slots, j, lane);
+    if (a.b < 0) return;  // a slot no batch needs (every thread of the CTA leaves here)
+    b = a.b;
+    k_in_batch = a.k;
+    const int raw = __ldg(p.seqlens_k + b);
+    L = min(max(raw, 0), p.Sk);
+    if (raw != L && k_in_batch == 0 && rg == 0 && hkv == 0 && threadIdx.x == 0) atomicOr(&g_error_word, kErrSeqlen);
+    tile_begin = k_in_batch * a.quota;
+    tile_end = min((L + kDecKeys - 1) / kDecKeys, tile_begin + a.quota);
+    coff = (p.causal == 2) ? L - p.Sq : 0;
+  }
+  const int ntiles = max(0, tile_end - tile_begin);
+  const int bhkv = b * p.Hkv + hkv;  // K/V head row of the tensor maps
+
+  // Let the combine kernel (a programmatic dependent launch) be scheduled
+  // as soon as every CTA of this grid has started; it waits for this grid's
+  // completion before it reads anything.
+  grid_dependency_trigger();
   __syncthreads();
 
   if (warp == kDecProducerWarp) {
     if (lane == 0 && ntiles > 0 && !p.withhold_loads) {
-      tma_prefetch_desc(&p.tm_k);
-      tma_prefetch_desc(&p.tm_v);
       int issued = 0;
       for (int it = 0; it < ntiles; ++it) {
         const int st = it % NSTAGE;
@@ -362,8 +489,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
         L += wt[w] * lw;
       }
       const float inv = (L > 0.f) ? 1.f / L : 0.f;
-      const int64_t row = row_base + lr;
-      float* dst = p.part_o + (row * p.nsplit + split) * D + c0;
+      // partial row [kv head][slot][local row]
+      const int64_t pr = (static_cast<int64_t>(hkv) * slots + j) * rows_total + lr;
+      float* dst = p.part_o + pr * D + c0;
 #pragma unroll
       for (int cc = 0; cc < kCols; cc += 4) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -382,7 +510,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
         *reinterpret_cast<float4*>(dst + cc) = acc;
       }
       if ((threadIdx.x & 7) == 0)
-        p.part_ml[row * p.nsplit + split] = make_float2(L > 0.f ? M * p.scale : -INFINITY, L);
+        p.part_ml[pr] = make_float2(L > 0.f ? M * p.scale : -INFINITY, L);
     }
   }
 }
@@ -398,31 +526,55 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
 // The kernel is launched as a programmatic dependent of the split kernel: it
 // may start while the split kernel's last CTAs run, and waits for that
 // grid's completion (and the visibility of its writes) before reading.
-// Where output row (b*Hq + h)*Sq + i lives: b*sb + h*sh + i*sr elements.
-struct RowLayout {
-  int Hq, Sq;
+struct CombineParams {
+  const float* part_o;     // as DecodeParams
+  const float2* part_ml;
+  const int* seqlens_k;    // per-batch lengths (the slot deal of the split kernel), or nullptr:
+                           // nsplit slots from b * nsplit
+  uint16_t* out;           // output row (b*Hq + h)*Sq + i at b*sb + h*sh + i*sr elements
+  float* lse;              // [B*Hq*Sq] or nullptr
+  int64_t rows;            // B*Hq*Sq
+  int B, Hq, Sq, Sk, group, nsplit, slots;
   int64_t sb, sh, sr;
 };
 
 template <int D>
-__global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ part_o,
-                                                             const float2* __restrict__ part_ml,
-                                                             uint16_t* __restrict__ out, float* __restrict__ lse,
-                                                             int64_t rows, int nsplit, RowLayout ol) {
+__global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_constant__ CombineParams cp) {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   constexpr int kPer = D / 32;  // floats per lane: 4 (one 16-byte load) or 2
   constexpr int kUnroll = 8;
   constexpr float kLog2e = 1.4426950408889634f;
   // the next kernel in the stream (a programmatic dependent) may be scheduled now
   grid_dependency_trigger();
-  grid_dependency_wait();
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const float2* ml = part_ml + row * nsplit;
+  if (row >= cp.rows) {
+    grid_dependency_wait();
+    return;
+  }
+  const int64_t bh = row / cp.Sq;
+  const int i = static_cast<int>(row - bh * cp.Sq);
+  const int b = static_cast<int>(bh / cp.Hq);
+  const int hq = static_cast<int>(bh - static_cast<int64_t>(b) * cp.Hq);
+  const int hkv = hq / cp.group;
+  const int rows_total = cp.group * cp.Sq;
+  const int lr = (hq - hkv * cp.group) * cp.Sq + i;  // row among the kv head's query rows
+  int first = b * cp.nsplit, nsplit = cp.nsplit;
+  if (cp.seqlens_k != nullptr) {
+    // Read before the wait: this grid starts only after every CTA of the
+    // split kernel has passed its own dependency wait, so whatever kernel
+    // wrote the lengths has completed and its writes are visible.
+    const int2 r = batch_slots(cp.seqlens_k, cp.B, cp.Sk, cp.slots, b, lane);
+    first = r.x;
+    nsplit = r.y;
+  }
+  grid_dependency_wait();
+  // partial rows of this output row: [kv head][slot][local row], slot stride rows_total
+  const int64_t pr0 = (static_cast<int64_t>(hkv) * cp.slots + first) * rows_total + lr;
+  const int64_t pstride = rows_total;
   float M = -INFINITY;
   for (int s = lane; s < nsplit; s += 32) {
-    const float2 v = ml[s];
+    const float2 v = cp.part_ml[pr0 + s * pstride];
     if (v.y > 0.f) M = fmaxf(M, v.x);
   }
 #pragma unroll
@@ -432,12 +584,12 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
   float W = 0.f;
   if (M != -INFINITY) {
-    const float* po = part_o + row * nsplit * D + lane * kPer;
+    const float* po = cp.part_o + pr0 * D + lane * kPer;
     for (int s0 = 0; s0 < nsplit; s0 += 32) {
       const int n = min(32, nsplit - s0);
       float w_lane = 0.f;
       if (lane < n) {
-        const float2 v = ml[s0 + lane];
+        const float2 v = cp.part_ml[pr0 + (s0 + lane) * pstride];
         w_lane = (v.y > 0.f) ? v.y * ex2_approx((v.x - M) * kLog2e) : 0.f;
       }
       W += w_lane;
@@ -446,7 +598,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
           if (i0 + u < n) {
-            const float* src = po + static_cast<int64_t>(s0 + i0 + u) * D;
+            const float* src = po + (s0 + i0 + u) * pstride * D;
             if constexpr (kPer == 4) {
               const float4 t = *reinterpret_cast<const float4*>(src);
               x[u][0] = t.x;
@@ -474,17 +626,15 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
     for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
   }
   const float inv = (W > 0.f) ? 1.f / W : 0.f;
-  const int64_t bh = row / ol.Sq;
-  const int64_t bb = bh / ol.Hq;
-  uint16_t* dst = out + bb * ol.sb + (bh - bb * ol.Hq) * ol.sh + (row - bh * ol.Sq) * ol.sr + lane * kPer;
+  uint16_t* dst = cp.out + b * cp.sb + hq * cp.sh + i * cp.sr + lane * kPer;
   if constexpr (kPer == 4) {
     *reinterpret_cast<uint2*>(dst) =
         make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
   } else {
     *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   }
-  if (lane == 0 && lse != nullptr)
-    lse[row] = (W > 0.f) ? M + lg2_approx(W) * 0.69314718055994531f : -INFINITY;
+  if (lane == 0 && cp.lse != nullptr)
+    cp.lse[row] = (W > 0.f) ? M + lg2_approx(W) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace sdpa

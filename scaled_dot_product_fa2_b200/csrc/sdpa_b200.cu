@@ -327,6 +327,8 @@ bool decode_shape(int B, int Hq, int Hkv, int Sq, int Sk, int d, int num_splits,
   return true;
 }
 
+// Workspace: fp32 partial outputs and (max, sum) pairs of every (kv head,
+// slot, query row).
 size_t decode_ws_bytes(int B, int Hq, int Sq, int d, int nsplit) {
   const size_t rows = static_cast<size_t>(B) * Hq * Sq;
   const size_t po = rows * nsplit * d * sizeof(float);
@@ -334,8 +336,8 @@ size_t decode_ws_bytes(int B, int Hq, int Sq, int d, int nsplit) {
 }
 
 template <int D>
-attn_status_t launch_decode(const DecodeParams& prm, int grid, float* part_o, float2* part_ml, void* o, float* lse,
-                            int64_t rows, int dev, cudaStream_t st) {
+attn_status_t launch_decode(const DecodeParams& prm, int grid, void* o, float* lse, int64_t rows, int dev,
+                            cudaStream_t st) {
   static bool smem_done[kMaxDevices] = {};
   static std::mutex mu;
   using Cfg = DecodeCfg<D, kDecStages>;
@@ -371,13 +373,25 @@ attn_status_t launch_decode(const DecodeParams& prm, int grid, float* part_o, fl
   ccfg.stream = st;
   ccfg.attrs = attr;
   ccfg.numAttrs = 1;
+  CombineParams cp;
+  cp.part_o = prm.part_o;
+  cp.part_ml = prm.part_ml;
+  cp.seqlens_k = prm.seqlens_k;
+  cp.out = static_cast<uint16_t*>(o);
+  cp.lse = lse;
+  cp.rows = rows;
+  cp.B = prm.B;
+  cp.Hq = prm.Hq;
+  cp.Sq = prm.Sq;
+  cp.Sk = prm.Sk;
+  cp.group = prm.group;
+  cp.nsplit = prm.nsplit;
+  cp.slots = prm.B * prm.nsplit;
   // q and o share the layout (q's strides are the caller's choice of layout)
-  const RowLayout ol = {prm.Hq, prm.Sq, prm.q_sb, prm.q_sh, prm.q_sr};
-  return cudaLaunchKernelEx(&ccfg, decode_combine_kernel<D>, static_cast<const float*>(part_o),
-                            static_cast<const float2*>(part_ml), static_cast<uint16_t*>(o), lse, rows,
-                            prm.nsplit, ol) == cudaSuccess
-             ? ATTN_OK
-             : ATTN_ERR_CUDA;
+  cp.sb = prm.q_sb;
+  cp.sh = prm.q_sh;
+  cp.sr = prm.q_sr;
+  return cudaLaunchKernelEx(&ccfg, decode_combine_kernel<D>, cp) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 // The three backward kernels, in stream order: prep (D, LSE in log2), then
@@ -585,8 +599,9 @@ static attn_status_t decode_impl(const void* q, const void* k_cache, const void*
   if (!make_map(&prm.tm_k, k_cache, d, Sk, static_cast<int64_t>(B) * Hkv, kDecKeys) ||
       !make_map(&prm.tm_v, v_cache, d, Sk, static_cast<int64_t>(B) * Hkv, kDecKeys))
     return ATTN_ERR_CUDA;
-  float* part_o = static_cast<float*>(workspace);
-  float2* part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + rows * ns * d * sizeof(float));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* part_o = reinterpret_cast<float*>(ws);
+  float2* part_ml = reinterpret_cast<float2*>(ws + rows * ns * d * sizeof(float));
   prm.q = static_cast<const uint16_t*>(q);
   const int layout = ex ? ex->layout : ATTN_LAYOUT_BHSD;
   const Strides qs = layout_strides(layout, Hq, Sq, d);
@@ -617,8 +632,8 @@ static attn_status_t decode_impl(const void* q, const void* k_cache, const void*
   prm.withhold_loads = withhold_loads ? 1 : 0;
   const int64_t grid = static_cast<int64_t>(B) * Hkv * ns * rg;
   if (grid > INT_MAX || (rows + 3) / 4 > INT_MAX) return ATTN_ERR_SHAPE;
-  if (d == 128) return launch_decode<128>(prm, static_cast<int>(grid), part_o, part_ml, o, lse, rows, dev, st);
-  return launch_decode<64>(prm, static_cast<int>(grid), part_o, part_ml, o, lse, rows, dev, st);
+  if (d == 128) return launch_decode<128>(prm, static_cast<int>(grid), o, lse, rows, dev, st);
+  return launch_decode<64>(prm, static_cast<int>(grid), o, lse, rows, dev, st);
 }
 
 attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,

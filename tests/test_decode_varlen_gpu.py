@@ -130,10 +130,37 @@ SKEWED = [
 
 @pytest.mark.parametrize("lens,Hq,Hkv,Sq,cap", SKEWED, ids=["one_full", "b40", "two_row_groups", "many_pairs"])
 def test_varlen_skewed_length_mixes(sdpa, lens, Hq, Hkv, Sq, cap):
-    """Extreme mixes of per-batch lengths against the per-batch oracle."""
+    """Extreme mixes of per-batch lengths against the per-batch oracle, with the
+    automatic split count and with fixed ones (the slots of a kv head are dealt
+    to batches by their lengths, so the split count changes every batch's share)."""
     B = len(lens)
     q, k, v = parity.seeded(B, Hq, Hkv, Sq, cap, 128, seed=740 + B + Hq)
-    o, lse = run_varlen(sdpa, q, k, v, lens, BR)
-    sdpa.check_device_error()
     o_ref, lse_ref = per_batch_oracle(q, k, v, lens, 1 / math.sqrt(128), BR)
-    parity.compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, f"lens {lens[:4]}")
+    for splits in (0, 3, 16):
+        o, lse = run_varlen(sdpa, q, k, v, lens, BR, num_splits=splits)
+        sdpa.check_device_error()
+        parity.compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref,
+                       f"lens {lens[:4]} splits={splits}")
+
+
+def test_workspace_contents_do_not_matter(sdpa):
+    """Whatever the caller's workspace holds before a call (never written,
+    another call's leftovers) gives the same bits: the per-batch slot ranges and
+    the partials are written by the call before anything reads them."""
+    B, Hq, Hkv, Sq, cap = 6, 8, 2, 4, 1000
+    lens = [1000, 3, 0, 517, 64, 999]
+    q, k, v = parity.seeded(B, Hq, Hkv, Sq, cap, 128, seed=75)
+    qd, kd, vd = parity.to_dev(q, k, v)
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    ws = sdpa.decode_workspace(qd, kd)
+    results = []
+    for fill in (0x00, 0xFF, 0x5A, None, None):
+        if fill is not None:
+            ws.fill_(fill)
+        o, lse = sdpa.attn_decode_splitkv_varlen(qd, kd, vd, sl, causal=BR, workspace=ws)
+        results.append((o.clone(), lse.clone()))
+    sdpa.check_device_error()
+    for o, lse in results[1:]:
+        assert torch.equal(o, results[0][0]) and torch.equal(lse, results[0][1])
+    o_ref, lse_ref = per_batch_oracle(q, k, v, lens, 1 / math.sqrt(128), BR)
+    parity.compare(results[0][0].float().cpu().numpy(), results[0][1].cpu().numpy(), o_ref, lse_ref, "ws")
