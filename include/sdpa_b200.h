@@ -169,9 +169,9 @@ attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, const
 int attn_decode_num_splits(int B, int Hq, int Hkv, int Sq, int Sk, int d);
 
 /*
- * Bytes of workspace attn_decode_splitkv needs: fp32 partial outputs
- * [B*Hq*Sq][splits][d] plus fp32 (max, sum) pairs [B*Hq*Sq][splits], with
- * `splits` the effective split count for num_splits (0 = automatic).
+ * Bytes of workspace attn_decode_splitkv needs: B*Hq*Sq*splits fp32 partial
+ * output rows of d values plus as many fp32 (max, sum) pairs, with `splits`
+ * the effective split count for num_splits (0 = automatic).
  * Returns 0 for an invalid shape.
  */
 size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int d, int num_splits);
@@ -217,9 +217,12 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
  *                     batch b sees key j iff j <= i + seqlens_k[b] - Sq.
  * The grid, the split count and the workspace size depend only on
  * Sk_capacity (attn_decode_workspace_size(B, Hq, Hkv, Sq, Sk_capacity, d,
- * num_splits)); each batch's valid tiles are spread evenly over the splits on
- * the device.  A batch with length 0 (or a row that sees no key) gets o = 0
- * and lse = -inf.  Everything else is as for attn_decode_splitkv.
+ * num_splits)).  On the device, the B * splits CTAs of each kv head are dealt
+ * to the batches in proportion to their valid 64-key tiles (every batch gets
+ * at least one; the per-CTA tile count is the smallest that lets the deal
+ * fit), so a mix of long and short caches keeps the CTAs' work about equal.
+ * A batch with length 0 (or a row that sees no key) gets o = 0 and
+ * lse = -inf.  Everything else is as for attn_decode_splitkv.
  */
 attn_status_t attn_decode_splitkv_varlen(const void* q, const void* k_cache, const void* v_cache,
                                          const int* seqlens_k, void* o, float* lse, int B, int Hq, int Hkv, int Sq,
