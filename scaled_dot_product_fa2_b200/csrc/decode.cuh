@@ -521,8 +521,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
 // all empty gets O = 0 and LSE = -inf.
 //
 // Lane s of the warp holds split s's weight (32 splits at a time); the
-// partial rows are then read kUnroll splits at a time with independent
-// 16-byte loads, so a row costs a few memory latencies, not one per split.
+// partial rows are read kUnroll splits at a time with independent 16-byte
+// loads, and with up to 32 splits the first kUnroll of them are loaded with
+// the (max, sum) pairs, so a row of up to kUnroll splits costs one memory
+// latency.
 // The kernel is launched as a programmatic dependent of the split kernel: it
 // may start while the split kernel's last CTAs run, and waits for that
 // grid's completion (and the visibility of its writes) before reading.
@@ -572,58 +574,99 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
   // partial rows of this output row: [kv head][slot][local row], slot stride rows_total
   const int64_t pr0 = (static_cast<int64_t>(hkv) * cp.slots + first) * rows_total + lr;
   const int64_t pstride = rows_total;
+  const float* po = cp.part_o + pr0 * D + lane * kPer;
+  // lane's kPer columns of partial row s of this output row
+  auto load_part = [&](int s, float (&x)[kPer]) {
+    const float* src = po + s * pstride * D;
+    if constexpr (kPer == 4) {
+      const float4 t = *reinterpret_cast<const float4*>(src);
+      x[0] = t.x;
+      x[1] = t.y;
+      x[2] = t.z;
+      x[3] = t.w;
+    } else {
+      const float2 t = *reinterpret_cast<const float2*>(src);
+      x[0] = t.x;
+      x[1] = t.y;
+    }
+  };
   float M = -INFINITY;
-  for (int s = lane; s < nsplit; s += 32) {
-    const float2 v = cp.part_ml[pr0 + s * pstride];
-    if (v.y > 0.f) M = fmaxf(M, v.x);
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
   float W = 0.f;
-  if (M != -INFINITY) {
-    const float* po = cp.part_o + pr0 * D + lane * kPer;
-    for (int s0 = 0; s0 < nsplit; s0 += 32) {
-      const int n = min(32, nsplit - s0);
-      float w_lane = 0.f;
-      if (lane < n) {
-        const float2 v = cp.part_ml[pr0 + (s0 + lane) * pstride];
-        w_lane = (v.y > 0.f) ? v.y * ex2_approx((v.x - M) * kLog2e) : 0.f;
-      }
-      W += w_lane;
-      for (int i0 = 0; i0 < n; i0 += kUnroll) {
-        float x[kUnroll][kPer];
+  if (nsplit <= 32) {
+    // One round trip: lane s's (m_s, l_s) and the first kUnroll partial rows
+    // are loaded together, before the maximum is known.
+    const float2 v = (lane < nsplit) ? cp.part_ml[pr0 + lane * pstride] : make_float2(-INFINITY, 0.f);
+    float x[kUnroll][kPer];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          if (i0 + u < n) {
-            const float* src = po + (s0 + i0 + u) * pstride * D;
-            if constexpr (kPer == 4) {
-              const float4 t = *reinterpret_cast<const float4*>(src);
-              x[u][0] = t.x;
-              x[u][1] = t.y;
-              x[u][2] = t.z;
-              x[u][3] = t.w;
-            } else {
-              const float2 t = *reinterpret_cast<const float2*>(src);
-              x[u][0] = t.x;
-              x[u][1] = t.y;
-            }
-          }
+    for (int u = 0; u < kUnroll; ++u)
+      if (u < nsplit) load_part(u, x[u]);
+    M = (v.y > 0.f) ? v.x : -INFINITY;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if (M != -INFINITY) {
+      const float w_lane = (v.y > 0.f) ? v.y * ex2_approx((v.x - M) * kLog2e) : 0.f;
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const float w = __shfl_sync(0xffffffffu, w_lane, u);
+        if (u < nsplit) {
+#pragma unroll
+          for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w, x[u][e], acc[e]);
         }
+      }
+      for (int i0 = kUnroll; i0 < nsplit; i0 += kUnroll) {
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+          if (i0 + u < nsplit) load_part(i0 + u, x[u]);
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
           const float w = __shfl_sync(0xffffffffu, w_lane, (i0 + u) & 31);
-          if (i0 + u < n) {
+          if (i0 + u < nsplit) {
 #pragma unroll
             for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w, x[u][e], acc[e]);
           }
         }
       }
+      W = w_lane;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
+    }
+  } else {
+    for (int s = lane; s < nsplit; s += 32) {
+      const float2 v = cp.part_ml[pr0 + s * pstride];
+      if (v.y > 0.f) M = fmaxf(M, v.x);
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if (M != -INFINITY) {
+      for (int s0 = 0; s0 < nsplit; s0 += 32) {
+        const int n = min(32, nsplit - s0);
+        float w_lane = 0.f;
+        if (lane < n) {
+          const float2 v = cp.part_ml[pr0 + (s0 + lane) * pstride];
+          w_lane = (v.y > 0.f) ? v.y * ex2_approx((v.x - M) * kLog2e) : 0.f;
+        }
+        W += w_lane;
+        for (int i0 = 0; i0 < n; i0 += kUnroll) {
+          float x[kUnroll][kPer];
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u)
+            if (i0 + u < n) load_part(s0 + i0 + u, x[u]);
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u) {
+            const float w = __shfl_sync(0xffffffffu, w_lane, (i0 + u) & 31);
+            if (i0 + u < n) {
+#pragma unroll
+              for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w, x[u][e], acc[e]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
+    }
   }
   const float inv = (W > 0.f) ? 1.f / W : 0.f;
   uint16_t* dst = cp.out + b * cp.sb + hq * cp.sh + i * cp.sr + lane * kPer;
