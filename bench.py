@@ -694,6 +694,10 @@ def run_profile_case(args):
     elif args.profile == inputs.PREFILL_VARLEN.name:
         w = inputs.PREFILL_VARLEN
         runner = GpuPrefillVarlen(w, 0)
+    elif args.profile.endswith("_varlen"):
+        # a decode workload over its seeded per-batch lengths, e.g. decode_sq4_varlen
+        w = inputs.BY_NAME[args.profile[:-len("_varlen")]]
+        runner = GpuDecodeVarlen(w, 0)
     elif args.profile.endswith("_bias"):
         # a prefill workload with the [1, 1, S, S] bias, e.g. prefill_noncausal_s2048_bias
         w = inputs.BY_NAME[args.profile[:-len("_bias")]]

@@ -139,11 +139,14 @@ __device__ __forceinline__ int slot_quota(const int* __restrict__ seqlens, int B
   tot = warp_sum_i64(tot);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  // For q >= ceil(tot / slots) the slot count is at most B + slots < 2^32.
   auto fits = [&](int q) {
-    int64_t n = 0;
+    unsigned n = 0;
     for (int b0 = 0; b0 < B; b0 += 32)
-      if (b0 + lane < B) n += max(1, (tiles_at(b0) + q - 1) / q);
-    return warp_sum_i64(n) <= slots;
+      if (b0 + lane < B) n += static_cast<unsigned>(max(1, (tiles_at(b0) + q - 1) / q));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) n += __shfl_xor_sync(0xffffffffu, n, off);
+    return n <= static_cast<unsigned>(slots);
   };
   // No q below ceil(tot / slots) fits; q = max T_b always does (B <= slots),
   // and so does ceil(tot / (slots - B)), since max(1, ceil(T_b / q)) <= T_b / q + 1.
@@ -232,6 +235,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
   }
+  __syncthreads();  // the barriers are initialised; no CTA-wide barrier follows the length deal
   // Launched as a programmatic dependent of the previous kernel in the
   // stream (the previous call's combine, in a decode loop): this grid's CTAs
   // may be resident before that kernel ends, and wait here, before any global
@@ -276,7 +280,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
   // as soon as every CTA of this grid has started; it waits for this grid's
   // completion before it reads anything.
   grid_dependency_trigger();
-  __syncthreads();
 
   if (warp == kDecProducerWarp) {
     if (lane == 0 && ntiles > 0 && !p.withhold_loads) {
