@@ -582,6 +582,7 @@ def main():
 
 
 def measure_breakdown(flush, peak_tf, hbm_gbs, rank, reps: int = 10):
+    import scaled_dot_product_fa2_b200 as sdpa
     out = {}
     # the tiny causal workload (B=1, H=2, S=128, d=64): a launch-latency figure
     s = GpuPrefill(inputs.TINY, rank)
@@ -631,7 +632,7 @@ def measure_breakdown(flush, peak_tf, hbm_gbs, rank, reps: int = 10):
         ms = statistics.median(timed_calls([batch], slack_only, reps, 2)[0]) / DECODE_BATCH
         gbs = w.decode_bytes() / ms / 1e6
         out[w.name] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4),
-                       "splits": int(s.ws.numel() // (w.B * w.Hq * w.Sq * (w.d + 2) * 4)),
+                       "splits": sdpa.decode_num_splits(w.B, w.Hq, w.Hkv, w.Sq, w.Sk, w.d),
                        "launches_per_call": 2}
         del s
     for w in inputs.DECODE:
