@@ -217,10 +217,12 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
  *                     batch b sees key j iff j <= i + seqlens_k[b] - Sq.
  * The grid, the split count and the workspace size depend only on
  * Sk_capacity (attn_decode_workspace_size(B, Hq, Hkv, Sq, Sk_capacity, d,
- * num_splits)).  On the device, the B * splits CTAs of each kv head are dealt
- * to the batches in proportion to their valid 64-key tiles (every batch gets
- * at least one; the per-CTA tile count is the smallest that lets the deal
- * fit), so a mix of long and short caches keeps the CTAs' work about equal.
+ * num_splits)).  With more than one split and at most 128 batches, the
+ * B * splits CTAs of each kv head are dealt on the device to the batches in
+ * proportion to their valid 64-key tiles (every batch gets at least one; the
+ * per-CTA tile count is the smallest that lets the deal fit), so a mix of
+ * long and short caches keeps the CTAs' work about equal; otherwise each
+ * batch's valid tiles are spread evenly over its own splits.
  * A batch with length 0 (or a row that sees no key) gets o = 0 and
  * lse = -inf.  Everything else is as for attn_decode_splitkv.
  */

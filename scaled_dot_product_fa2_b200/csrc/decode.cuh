@@ -109,11 +109,13 @@ __device__ __forceinline__ int len_tiles(const int* __restrict__ seqlens, int bb
   return bb < B ? (min(max(__ldg(seqlens + bb), 0), Sk) + kDecKeys - 1) / kDecKeys : 0;
 }
 
-__device__ __forceinline__ int64_t warp_sum_i64(int64_t v) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-  return v;
-}
+// The deal holds the tile counts of up to kDealMaxBatch batches in registers
+// (kDealChunks per lane); with more batches, or one split, each batch keeps
+// nsplit CTAs and its tiles are spread evenly over them.
+constexpr int kDealChunks = 4;
+constexpr int kDealMaxBatch = 32 * kDealChunks;
+
+__device__ __forceinline__ bool use_deal(int B, int nsplit) { return nsplit > 1 && B <= kDealMaxBatch; }
 
 // Inclusive prefix sum over the warp.
 __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
@@ -125,25 +127,31 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
   return v;
 }
 
-// The quota q.  t0 = len_tiles(lane): the first 32 batches stay in a register.
+// Tile counts of batches c*32 + lane (0 beyond B), and the quota q.
+struct DealTiles {
+  int t[kDealChunks];
+};
+
 __device__ __forceinline__ int slot_quota(const int* __restrict__ seqlens, int B, int Sk, int slots, int lane,
-                                          int t0) {
-  auto tiles_at = [&](int b0) { return b0 == 0 ? t0 : len_tiles(seqlens, b0 + lane, B, Sk); };
+                                          DealTiles& dt) {
   int64_t tot = 0;
   int mx = 0;
-  for (int b0 = 0; b0 < B; b0 += 32) {
-    const int t = tiles_at(b0);
-    tot += t;
-    mx = max(mx, t);
+#pragma unroll
+  for (int c = 0; c < kDealChunks; ++c) {
+    dt.t[c] = len_tiles(seqlens, c * 32 + lane, B, Sk);
+    tot += dt.t[c];
+    mx = max(mx, dt.t[c]);
   }
-  tot = warp_sum_i64(tot);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   // For q >= ceil(tot / slots) the slot count is at most B + slots < 2^32.
   auto fits = [&](int q) {
     unsigned n = 0;
-    for (int b0 = 0; b0 < B; b0 += 32)
-      if (b0 + lane < B) n += static_cast<unsigned>(max(1, (tiles_at(b0) + q - 1) / q));
+#pragma unroll
+    for (int c = 0; c < kDealChunks; ++c)
+      if (c * 32 + lane < B) n += static_cast<unsigned>(max(1, (dt.t[c] + q - 1) / q));
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) n += __shfl_xor_sync(0xffffffffu, n, off);
     return n <= static_cast<unsigned>(slots);
@@ -169,38 +177,39 @@ struct SlotAssign {
   int b, k, quota;  // b = -1: a slot that no batch needs
 };
 
+// Requires use_deal(B, nsplit).
 __device__ __forceinline__ SlotAssign assign_slot(const int* __restrict__ seqlens, int B, int Sk, int slots, int j,
                                                   int lane) {
-  const int t0 = len_tiles(seqlens, lane, B, Sk);
-  const int q = slot_quota(seqlens, B, Sk, slots, lane, t0);
+  DealTiles dt;
+  const int q = slot_quota(seqlens, B, Sk, slots, lane, dt);
   int start = 0;
-  for (int b0 = 0; b0 < B; b0 += 32) {
-    const int t = b0 == 0 ? t0 : len_tiles(seqlens, b0 + lane, B, Sk);
-    const int n = (b0 + lane < B) ? max(1, (t + q - 1) / q) : 0;
+#pragma unroll
+  for (int c = 0; c < kDealChunks; ++c) {
+    const int n = (c * 32 + lane < B) ? max(1, (dt.t[c] + q - 1) / q) : 0;
     const int incl = warp_incl_scan(n, lane);
     const int excl = incl - n;
     const unsigned hit = __ballot_sync(0xffffffffu, n > 0 && j >= start + excl && j < start + incl);
     if (hit != 0u) {
       const int src = __ffs(hit) - 1;
-      return {b0 + src, j - start - __shfl_sync(0xffffffffu, excl, src), q};
+      return {c * 32 + src, j - start - __shfl_sync(0xffffffffu, excl, src), q};
     }
     start += __shfl_sync(0xffffffffu, incl, 31);
   }
   return {-1, 0, q};
 }
 
-// (first slot, slot count) of batch b.
+// (first slot, slot count) of batch b.  Requires use_deal(B, nsplit).
 __device__ __forceinline__ int2 batch_slots(const int* __restrict__ seqlens, int B, int Sk, int slots, int b,
                                             int lane) {
-  const int t0 = len_tiles(seqlens, lane, B, Sk);
-  const int q = slot_quota(seqlens, B, Sk, slots, lane, t0);
+  DealTiles dt;
+  const int q = slot_quota(seqlens, B, Sk, slots, lane, dt);
   int start = 0;
-  for (int b0 = 0; b0 < B; b0 += 32) {
-    const int t = b0 == 0 ? t0 : len_tiles(seqlens, b0 + lane, B, Sk);
-    const int n = (b0 + lane < B) ? max(1, (t + q - 1) / q) : 0;
+#pragma unroll
+  for (int c = 0; c < kDealChunks; ++c) {
+    const int n = (c * 32 + lane < B) ? max(1, (dt.t[c] + q - 1) / q) : 0;
     const int incl = warp_incl_scan(n, lane);
-    if (b < b0 + 32) {
-      const int src = b - b0;
+    if (b < c * 32 + 32) {
+      const int src = b - c * 32;
       return make_int2(start + __shfl_sync(0xffffffffu, incl - n, src), __shfl_sync(0xffffffffu, n, src));
     }
     start += __shfl_sync(0xffffffffu, incl, 31);
@@ -262,15 +271,25 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     tile_begin = k_in_batch * p.tiles_per_split;
     tile_end = min((L + kDecKeys - 1) / kDecKeys, tile_begin + p.tiles_per_split);
   } else {
-    const SlotAssign a = assign_slot(p.seqlens_k, p.B, p.Sk, slots, j, lane);
-    if (a.b < 0) return;  // a slot no batch needs (every thread of the CTA leaves here)
-    b = a.b;
-    k_in_batch = a.k;
+    int quota;
+    if (use_deal(p.B, p.nsplit)) {
+      const SlotAssign a = assign_slot(p.seqlens_k, p.B, p.Sk, slots, j, lane);
+      if (a.b < 0) return;  // a slot no batch needs (every thread of the CTA leaves here)
+      b = a.b;
+      k_in_batch = a.k;
+      quota = a.quota;
+    } else {
+      b = j / p.nsplit;
+      k_in_batch = j - b * p.nsplit;
+      quota = -1;
+    }
     const int raw = __ldg(p.seqlens_k + b);
     L = min(max(raw, 0), p.Sk);
     if (raw != L && k_in_batch == 0 && rg == 0 && hkv == 0 && threadIdx.x == 0) atomicOr(&g_error_word, kErrSeqlen);
-    tile_begin = k_in_batch * a.quota;
-    tile_end = min((L + kDecKeys - 1) / kDecKeys, tile_begin + a.quota);
+    const int tiles = (L + kDecKeys - 1) / kDecKeys;
+    if (quota < 0) quota = (tiles + p.nsplit - 1) / p.nsplit;
+    tile_begin = k_in_batch * quota;
+    tile_end = min(tiles, tile_begin + quota);
     coff = (p.causal == 2) ? L - p.Sq : 0;
   }
   const int ntiles = max(0, tile_end - tile_begin);
@@ -534,8 +553,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
 struct CombineParams {
   const float* part_o;     // as DecodeParams
   const float2* part_ml;
-  const int* seqlens_k;    // per-batch lengths (the slot deal of the split kernel), or nullptr:
-                           // nsplit slots from b * nsplit
+  const int* seqlens_k;    // per-batch lengths (the slot deal of the split kernel when
+                           // use_deal), or nullptr: nsplit slots from b * nsplit
   uint16_t* out;           // output row (b*Hq + h)*Sq + i at b*sb + h*sh + i*sr elements
   float* lse;              // [B*Hq*Sq] or nullptr
   int64_t rows;            // B*Hq*Sq
@@ -565,7 +584,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
   const int rows_total = cp.group * cp.Sq;
   const int lr = (hq - hkv * cp.group) * cp.Sq + i;  // row among the kv head's query rows
   int first = b * cp.nsplit, nsplit = cp.nsplit;
-  if (cp.seqlens_k != nullptr) {
+  if (cp.seqlens_k != nullptr && use_deal(cp.B, cp.nsplit)) {
     // Read before the wait: this grid starts only after every CTA of the
     // split kernel has passed its own dependency wait, so whatever kernel
     // wrote the lengths has completed and its writes are visible.

@@ -125,10 +125,13 @@ SKEWED = [
     ([5, 4000, 0, 8191, 64, 65, 1, 3000] * 5, 8, 2, 1, 8192),  # 40 batches of every kind of length
     ([300, 1, 299], 64, 2, 1, 300),                           # 32 query rows per kv head: two row groups
     ([2] * 200, 4, 4, 1, 64),                                 # 800 (batch, kv head) pairs, more than one wave
+    ([5, 2000, 0, 2047] * 32, 4, 1, 1, 2048),                 # 128 batches: the largest dealt batch count
+    ([7, 1000, 0, 513] * 40, 4, 1, 1, 1000),                  # 160 batches: tiles spread evenly per batch
 ]
 
 
-@pytest.mark.parametrize("lens,Hq,Hkv,Sq,cap", SKEWED, ids=["one_full", "b40", "two_row_groups", "many_pairs"])
+@pytest.mark.parametrize("lens,Hq,Hkv,Sq,cap", SKEWED,
+                         ids=["one_full", "b40", "two_row_groups", "many_pairs", "b128", "b160"])
 def test_varlen_skewed_length_mixes(sdpa, lens, Hq, Hkv, Sq, cap):
     """Extreme mixes of per-batch lengths against the per-batch oracle, with the
     automatic split count and with fixed ones (the slots of a kv head are dealt
