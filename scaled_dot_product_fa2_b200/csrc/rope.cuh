@@ -18,7 +18,9 @@
 // rows per pass, the block 8 times that, and every lane issues the loads of
 // kRopeUnroll passes before it uses any, to keep enough bytes in flight.  The
 // partner half of each rotated pair sits d/16 lanes away and comes over by
-// shuffle.
+// shuffle.  Tokens are pipelined one deep: a block issues the loads of its
+// next token's rows before it rotates and stores the current token's, so its
+// loads never wait for its stores (at 64 registers, four blocks per SM).
 #pragma once
 #include <climits>
 
@@ -86,67 +88,107 @@ __global__ void __launch_bounds__(kRopeWarps * 32, kRopeBlocksPerSm)
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.B; i += gridDim.x * blockDim.x)
     if (p.total_lens != nullptr) p.total_lens[i] = rope_total_length(__ldg(p.past_lens + i), p.S_new);
 
-  for (int bt = blockIdx.x; bt < p.tokens; bt += gridDim.x) {  // block-uniform
-    const int b = bt / p.S_new;
-    const int t = bt - b * p.S_new;
+  // Token bt's position, or -1 when it is out of range (reported, skipped).
+  auto token_pos = [&](int bt, int& b, int& t) {
+    b = bt / p.S_new;
+    t = bt - b * p.S_new;
     const int past = __ldg(p.past_lens + b);
     // pos = past + t must lie in [0, min(cap, max_pos)); tested without
     // forming past + t, which overflows for a corrupt past near INT_MAX
     if (past < 0 || past > p.cap - 1 - t || past > p.max_pos - 1 - t) {
       if (threadIdx.x == 0) atomicOr(&g_error_word, kErrSeqlen);
-      continue;
+      return -1;
     }
-    const int pos = past + t;
-    const float4* cr = reinterpret_cast<const float4*>(p.cos_t + static_cast<int64_t>(pos) * kHalf + i0);
-    const float4* sr = reinterpret_cast<const float4*>(p.sin_t + static_cast<int64_t>(pos) * kHalf + i0);
-    const float4 c0 = __ldg(cr), c1 = __ldg(cr + 1), s0 = __ldg(sr), s1 = __ldg(sr + 1);
-    const float c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-    const float s[8] = {s0.x * sign, s0.y * sign, s0.z * sign, s0.w * sign,
-                        s1.x * sign, s1.y * sign, s1.z * sign, s1.w * sign};
+    return past + t;
+  };
+  // The loads of one token's head rows (kRopeUnroll block passes cover every
+  // row when (Hq + 2 Hkv) <= kBlockRows * kRopeUnroll; more rows take further
+  // rounds in process_token).
+  auto load_rows = [&](int bt, int h0, uint4 (&x)[kRopeUnroll]) {
     const uint4* src = reinterpret_cast<const uint4*>(p.packed + static_cast<int64_t>(bt) * slots * D) + sub;
+#pragma unroll
+    for (int u = 0; u < kRopeUnroll; ++u) {
+      const int h = h0 + u * kBlockRows + row_in_block;
+      x[u] = h < slots ? __ldg(src + h * (D / 8)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  // Rotate and store the rows of one round.
+  auto store_rows = [&](int b, int t, int pos, int h0, const uint4 (&x)[kRopeUnroll], const float (&c)[8],
+                        const float (&s)[8]) {
     uint16_t* const q_base = p.q_out + b * p.q_sb + t * p.q_sr;
     const int64_t c_off = b * p.c_sb + static_cast<int64_t>(pos) * p.c_sr;
-
-    for (int h0 = 0; h0 < slots; h0 += kBlockRows * kRopeUnroll) {  // block-uniform
-      uint4 x[kRopeUnroll];
 #pragma unroll
-      for (int u = 0; u < kRopeUnroll; ++u) {
-        const int h = h0 + u * kBlockRows + row_in_block;
-        x[u] = h < slots ? __ldg(src + h * (D / 8)) : make_uint4(0u, 0u, 0u, 0u);
-      }
+    for (int u = 0; u < kRopeUnroll; ++u) {
+      // every lane of the warp takes part in the exchange; the partner lane
+      // always belongs to the same row
+      uint4 y;
+      y.x = __shfl_xor_sync(0xffffffffu, x[u].x, kPartner);
+      y.y = __shfl_xor_sync(0xffffffffu, x[u].y, kPartner);
+      y.z = __shfl_xor_sync(0xffffffffu, x[u].z, kPartner);
+      y.w = __shfl_xor_sync(0xffffffffu, x[u].w, kPartner);
+      const int h = h0 + u * kBlockRows + row_in_block;
+      if (h >= slots) continue;
+      uint4 out = x[u];
+      uint16_t* dst;
+      if (h < p.Hq + p.Hkv) {
+        dst = h < p.Hq ? q_base + h * p.q_sh : p.k_cache + c_off + (h - p.Hq) * p.c_sh;
+        const uint32_t xs[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+        const uint32_t ys[4] = {y.x, y.y, y.z, y.w};
+        uint32_t o[4];
 #pragma unroll
-      for (int u = 0; u < kRopeUnroll; ++u) {
-        // every lane of the warp takes part in the exchange; the partner lane
-        // always belongs to the same row
-        uint4 y;
-        y.x = __shfl_xor_sync(0xffffffffu, x[u].x, kPartner);
-        y.y = __shfl_xor_sync(0xffffffffu, x[u].y, kPartner);
-        y.z = __shfl_xor_sync(0xffffffffu, x[u].z, kPartner);
-        y.w = __shfl_xor_sync(0xffffffffu, x[u].w, kPartner);
-        const int h = h0 + u * kBlockRows + row_in_block;
-        if (h >= slots) continue;
-        uint4 out = x[u];
-        uint16_t* dst;
-        if (h < p.Hq + p.Hkv) {
-          dst = h < p.Hq ? q_base + h * p.q_sh : p.k_cache + c_off + (h - p.Hq) * p.c_sh;
-          const uint32_t xs[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
-          const uint32_t ys[4] = {y.x, y.y, y.z, y.w};
-          uint32_t o[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float xa = bf16_bits_to_float(static_cast<unsigned short>(xs[j] & 0xFFFFu));
-            const float xb = bf16_bits_to_float(static_cast<unsigned short>(xs[j] >> 16));
-            const float ya = bf16_bits_to_float(static_cast<unsigned short>(ys[j] & 0xFFFFu));
-            const float yb = bf16_bits_to_float(static_cast<unsigned short>(ys[j] >> 16));
-            o[j] = pack_bf16x2(fmaf(ya, s[2 * j], xa * c[2 * j]), fmaf(yb, s[2 * j + 1], xb * c[2 * j + 1]));
-          }
-          out = make_uint4(o[0], o[1], o[2], o[3]);
-        } else {
-          dst = p.v_cache + c_off + (h - p.Hq - p.Hkv) * p.c_sh;  // v: copied as is
+        for (int j = 0; j < 4; ++j) {
+          const float xa = bf16_bits_to_float(static_cast<unsigned short>(xs[j] & 0xFFFFu));
+          const float xb = bf16_bits_to_float(static_cast<unsigned short>(xs[j] >> 16));
+          const float ya = bf16_bits_to_float(static_cast<unsigned short>(ys[j] & 0xFFFFu));
+          const float yb = bf16_bits_to_float(static_cast<unsigned short>(ys[j] >> 16));
+          o[j] = pack_bf16x2(fmaf(ya, s[2 * j], xa * c[2 * j]), fmaf(yb, s[2 * j + 1], xb * c[2 * j + 1]));
         }
-        reinterpret_cast<uint4*>(dst)[sub] = out;
+        out = make_uint4(o[0], o[1], o[2], o[3]);
+      } else {
+        dst = p.v_cache + c_off + (h - p.Hq - p.Hkv) * p.c_sh;  // v: copied as is
+      }
+      reinterpret_cast<uint4*>(dst)[sub] = out;
+    }
+  };
+
+  // Tokens are pipelined one deep: the first round of the next token's rows
+  // is loaded before this token's rows are rotated and stored, so the loads
+  // of a block never stop for its stores.
+  int bt = blockIdx.x;  // block-uniform
+  if (bt >= p.tokens) return;
+  int b, t;
+  int pos = token_pos(bt, b, t);
+  uint4 x[kRopeUnroll];
+  if (pos >= 0) load_rows(bt, 0, x);
+  while (true) {
+    const int nbt = bt + gridDim.x;
+    int nb = 0, nt = 0, npos = -1;
+    uint4 xn[kRopeUnroll];
+    if (nbt < p.tokens) {
+      npos = token_pos(nbt, nb, nt);
+      if (npos >= 0) load_rows(nbt, 0, xn);
+    }
+    if (pos >= 0) {
+      const float4* cr = reinterpret_cast<const float4*>(p.cos_t + static_cast<int64_t>(pos) * kHalf + i0);
+      const float4* sr = reinterpret_cast<const float4*>(p.sin_t + static_cast<int64_t>(pos) * kHalf + i0);
+      const float4 c0 = __ldg(cr), c1 = __ldg(cr + 1), s0 = __ldg(sr), s1 = __ldg(sr + 1);
+      const float c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      const float s[8] = {s0.x * sign, s0.y * sign, s0.z * sign, s0.w * sign,
+                          s1.x * sign, s1.y * sign, s1.z * sign, s1.w * sign};
+      store_rows(b, t, pos, 0, x, c, s);
+      for (int h0 = kBlockRows * kRopeUnroll; h0 < slots; h0 += kBlockRows * kRopeUnroll) {  // block-uniform
+        uint4 xr[kRopeUnroll];
+        load_rows(bt, h0, xr);
+        store_rows(b, t, pos, h0, xr, c, s);
       }
     }
+    if (nbt >= p.tokens) break;
+    bt = nbt;
+    b = nb;
+    t = nt;
+    pos = npos;
+#pragma unroll
+    for (int u = 0; u < kRopeUnroll; ++u) x[u] = xn[u];
   }
 }
 
