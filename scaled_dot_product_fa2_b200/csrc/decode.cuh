@@ -15,16 +15,18 @@
 //     warp; K/V tiles of 64 keys stream through an NSTAGE-deep ring of
 //     128-byte-swizzled shared-memory tiles.
 //   * A KV head has B * nsplit slots (CTAs).  With one cache length every
-//     batch takes nsplit of them; with per-batch lengths the slots are dealt
-//     in proportion to each batch's tiles (assign_slot), so a mix of long and
-//     short caches keeps every CTA's share of the keys about equal.
+//     batch takes nsplit of them; with per-batch lengths (several splits, at
+//     most kDealMaxBatch batches) the slots are dealt in proportion to each
+//     batch's tiles (assign_slot), so a mix of long and short caches keeps
+//     every CTA's share of the keys about equal.
 //   * The work per byte is tiny (<= 16 query rows), so the contraction runs on
 //     warp-level mma.sync m16n8k16 (bf16, fp32 accumulate): the kernel is
 //     bound by HBM bandwidth, not by the tensor pipe.  Each warp owns 16 keys
 //     of every tile and its own running (m, l, O); the four warps merge once
 //     through shared memory at the end.
 //   * The combine kernel is one warp per output row with 16-byte coalesced
-//     loads of the fp32 partials.
+//     loads of the fp32 partials, the (max, sum) pairs loaded with the first
+//     eight partial rows; it is a programmatic dependent of the split kernel.
 #pragma once
 #include "ptx.cuh"
 
