@@ -70,6 +70,22 @@ constexpr int kBwdComputeWarps = 8;
 constexpr int kBwdMmaWarp = 8;
 constexpr int kBwdLoadWarp = 9;
 constexpr int kBwdStages = 2;
+constexpr int kBwdHeadGroup = 8;  // heads dealt together under a causal mask (see lpt_coords)
+
+// Under a causal mask the CTAs' work differs up to n-fold (a key tile near
+// the start is seen by every query tile, one near the end by few), and CTAs
+// are dispatched in blockIdx order: in head-major order the heaviest tiles of
+// the last heads would start last and run on alone.  So CTA idx takes, within
+// groups of kBwdHeadGroup heads (whose K, V, Q and dO stay in L2 together),
+// the tiles heaviest first: rank 0 = heaviest.  Covers [0, n_t * heads).
+__device__ __forceinline__ void lpt_coords(int idx, int n_t, int heads, int& rank, int& head) {
+  const int per_group = n_t * kBwdHeadGroup;
+  const int g = idx / per_group;
+  const int rem = idx - g * per_group;
+  const int gh = min(kBwdHeadGroup, heads - g * kBwdHeadGroup);
+  rank = rem / gh;
+  head = g * kBwdHeadGroup + (rem - rank * gh);
+}
 constexpr float kLog2e = 1.4426950408889634f;
 
 // 1-D bulk copy global -> shared (no tensor map), completion counted on `bar`.
@@ -216,8 +232,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int kt = static_cast<int>(blockIdx.x % p.n_kt);
-  const int bkv = static_cast<int>(blockIdx.x / p.n_kt);
+  int kt, bkv;
+  if (p.causal) {
+    lpt_coords(static_cast<int>(blockIdx.x), p.n_kt, p.B * p.Hkv, kt, bkv);  // early key tiles are heaviest
+  } else {
+    kt = static_cast<int>(blockIdx.x % p.n_kt);
+    bkv = static_cast<int>(blockIdx.x / p.n_kt);
+  }
   const int b = bkv / p.Hkv;
   const int hkv = bkv - b * p.Hkv;
   const int k0 = kt * 128;
@@ -472,8 +493,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qt = static_cast<int>(blockIdx.x % p.n_qt);
-  const int bh = static_cast<int>(blockIdx.x / p.n_qt);
+  int qt, bh;
+  if (p.causal) {
+    int rank;
+    lpt_coords(static_cast<int>(blockIdx.x), p.n_qt, p.B * p.Hq, rank, bh);
+    qt = p.n_qt - 1 - rank;  // late query tiles are heaviest
+  } else {
+    qt = static_cast<int>(blockIdx.x % p.n_qt);
+    bh = static_cast<int>(blockIdx.x / p.n_qt);
+  }
   const int b = bh / p.Hq;
   const int hq = bh - b * p.Hq;
   const int hkv = hq / p.group;
