@@ -286,12 +286,14 @@ class GpuPrefill:
         import scaled_dot_product_fa2_b200 as sdpa
         sdpa.attn_fwd(self.q, self.k, self.v, causal=self.w.causal, scale=self.w.scale, out=self.o, lse=self.lse)
 
-    def run_e2e(self):
-        import scaled_dot_product_fa2_b200 as sdpa
+    def copy_inputs(self):
+        """q, k, v from pinned host memory, on the current stream."""
         self.q.copy_(self.host[0], non_blocking=True)
         self.k.copy_(self.host[1], non_blocking=True)
         self.v.copy_(self.host[2], non_blocking=True)
-        sdpa.attn_fwd(self.q, self.k, self.v, causal=self.w.causal, scale=self.w.scale, out=self.o, lse=self.lse)
+
+    def copy_outputs(self):
+        """o and lse back to pinned host memory, on the current stream."""
         self.o_host.copy_(self.o, non_blocking=True)
         self.lse_host.copy_(self.lse, non_blocking=True)
 
@@ -507,18 +509,47 @@ def main():
     ms_per_step = kernel_ms / args.steps
     value = weak_scaling_value(world, flops_step, args.steps, kernel_ms)
 
-    # ---- end to end through the public API with host buffers (pinned), same metric
-    for _ in range(2):
-        for s in shapes:
-            s.run_e2e()
+    # ---- end to end through the public API with host buffers (pinned), same metric.
+    # Every step copies each shape's q, k, v in, runs the forward and reads o
+    # and lse back, as a serving loop would: the input copies, the forwards and
+    # the read-backs go to three streams, so the two copy directions and the
+    # compute of different shapes overlap (each shape's buffers are reused only
+    # after their previous forward and read-back are done).
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in shapes]    # inputs of shape i on the device
+    ev_fwd = [torch.cuda.Event() for _ in shapes]   # forward of shape i done (inputs free, outputs ready)
+    ev_out = [torch.cuda.Event() for _ in shapes]   # outputs of shape i read back (outputs free)
+
+    def e2e_step(first: bool):
+        for i, s in enumerate(shapes):
+            with torch.cuda.stream(h2d_s):
+                if not first:
+                    h2d_s.wait_event(ev_fwd[i])
+                s.copy_inputs()
+                ev_in[i].record(h2d_s)
+            stream.wait_event(ev_in[i])
+            if not first:
+                stream.wait_event(ev_out[i])
+            s.run()
+            ev_fwd[i].record(stream)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev_fwd[i])
+                s.copy_outputs()
+                ev_out[i].record(d2h_s)
+
+    for it in range(2):
+        e2e_step(first=(it == 0))
     torch.cuda.synchronize()
     barrier(world)
     e_a = torch.cuda.Event(enable_timing=True)
     e_b = torch.cuda.Event(enable_timing=True)
     e_a.record(stream)
+    h2d_s.wait_event(e_a)
+    d2h_s.wait_event(e_a)
     for _ in range(args.steps):
-        for s in shapes:
-            s.run_e2e()
+        e2e_step(first=False)
+    stream.wait_stream(h2d_s)
+    stream.wait_stream(d2h_s)
     e_b.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(world, e_a.elapsed_time(e_b))
