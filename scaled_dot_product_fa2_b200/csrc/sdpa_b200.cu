@@ -517,10 +517,14 @@ static attn_status_t fwd_impl(const void* q, const void* k, const void* v, const
   prm.div_hq = make_fastdiv(static_cast<uint32_t>(std::max(Hq, 1)));
   prm.div_group = make_fastdiv(static_cast<uint32_t>(std::max(prm.group, 1)));
   prm.div_units = make_fastdiv(static_cast<uint32_t>(std::max(prm.num_units, 1)));
-  // Fixed lengths: persistent grid, one CTA per SM (the kernel's shared memory
-  // allows one).  Per-batch lengths: one CTA per unit, running CTAs take over
-  // the units of CTAs that have not started (see prefill.cuh).
-  prm.dynamic = (prm.seqlens_q != nullptr || prm.seqlens_k != nullptr) ? 1 : 0;
+  // Non-causal fixed lengths (units of equal cost): persistent grid, one CTA
+  // per SM (the kernel's shared memory allows one), units dealt statically.
+  // Per-batch lengths and causal masks (units of unequal cost): one CTA per
+  // unit, running CTAs take over the units of CTAs that have not started (see
+  // prefill.cuh), which balances the tail better than the static heaviest-
+  // first deal (measured on B200: causal seq 512 / 1024 / 2048 / 4096
+  // +4.0 / +5.8 / +0.8 / +0.3 %).
+  prm.dynamic = (prm.seqlens_q != nullptr || prm.seqlens_k != nullptr || causal != ATTN_CAUSAL_NONE) ? 1 : 0;
   const int64_t grid = prm.dynamic ? units : std::min<int64_t>(units, sms);
   if (d == 128) {
     return has_bias ? launch_prefill<128, kStagesD128Bias, true>(prm, static_cast<int>(grid), dev, st)
