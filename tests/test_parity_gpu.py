@@ -61,7 +61,8 @@ SMALL = [
     (1, 2, 2, 1, 1000, 128, BR),       # one query at the end of 1000 keys
     (3, 2, 2, 7, 129, 128, NONE),      # ragged both ways, tiny
     (1, 1, 1, 1024, 1024, 128, TL),    # 4 units, exercises LPT ordering
-    (4, 40, 8, 520, 520, 128, TL),     # 480 units > 148 CTAs: several dealing rounds, GQA group 5
+    (4, 40, 8, 520, 520, 128, TL),     # 480 units > 148 CTAs, one CTA per unit taken over at run time, GQA group 5
+    (4, 40, 8, 520, 520, 128, NONE),   # 480 units over the 148-CTA persistent grid: several dealing rounds
     (3, 32, 32, 300, 700, 64, BR),     # 192 units > 148 CTAs at d = 64 (8-slot ring)
 ]
 
@@ -151,8 +152,9 @@ def run_full_size(sdpa, w):
 @pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
 def test_prefill_full_size_every_tile_sampled(sdpa, w):
     """One oracle row inside every 128-row query tile of every head, so every
-    work unit of the persistent schedule (all rounds of its snake dealing) is
-    checked against the oracle, not only a random handful."""
+    work unit is checked against the oracle, not only a random handful: all
+    rounds of the persistent grid's snake dealing (non-causal) and every unit
+    taken over at run time (causal, GQA)."""
     (q, k, v), o, lse = run_full_size(sdpa, w)
     rows = parity.tile_rows(w.B, w.Hq, w.Sq, seed=w.seed)
     o_ref, lse_ref = parity.oracle_rows(q, k, v, w.eff_scale, w.causal, rows)
@@ -167,10 +169,11 @@ WHOLE = [inputs.BY_NAME["prefill_causal_s2048"], inputs.BY_NAME["prefill_noncaus
 
 @pytest.mark.parametrize("w", WHOLE, ids=lambda w: w.name)
 def test_prefill_whole_workload_element_by_element(sdpa, w):
-    """Every element of a whole benchmark workload against the oracle: 1024
-    work units over the 148-CTA persistent grid, so the multi-round snake
-    dealing and the ring and barrier phases that run on across units are
-    checked on every row."""
+    """Every element of a whole benchmark workload against the oracle: causal
+    seq 2048 (1024 work units, one CTA per unit, units taken over at run time
+    by running CTAs) and non-causal seq 4096 (512 units over the 148-CTA
+    persistent grid: the multi-round snake dealing and the ring and barrier
+    phases that run on across units), checked on every row."""
     (q, k, v), o, lse = run_full_size(sdpa, w)
     o_ref, lse_ref = parity.oracle_full(q, k, v, w.eff_scale, w.causal)
     parity.compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, w.name)
