@@ -129,7 +129,7 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
   return v;
 }
 
-// Tile counts of batches c*32 + lane (0 beyond B), and the quota q.
+// Tile counts of batches c*32 + lane, c < kDealChunks (0 beyond B).
 struct DealTiles {
   int t[kDealChunks];
 };
